@@ -1,0 +1,85 @@
+"""fp64 CPU oracle for the attention forward pass.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py``, never by the product package.  It
+shares no code with the CUDA path; the only thing both sides use is the
+seeded input generator in ``seeded_inputs``.
+
+``attention_fwd`` returns, per (b, h) and query row i, the plain definition
+  S = scale * Q K^T (fp64), S[i, j] = -inf for j > i when causal,
+  P = row softmax of S,  O = P V,  LSE_i = ln sum_j exp(S[i, j])
+as in the FlashAttention section of the TileLang tutorial (fused forward over
+Q/K/V tiles, validated against scaled-dot-product attention, causal and
+non-causal).  Every function here is pinned by ``tests/test_oracle.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from .build import build as _build, library_path
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            _build()
+        lib = ctypes.CDLL(path)
+        lib.oracle_attention_fwd.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int64] * 4 + [
+            ctypes.c_int, ctypes.c_double, ctypes.c_int]
+        lib.oracle_attention_fwd.restype = ctypes.c_int
+        lib.oracle_attention_rows.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 4 + [
+            ctypes.c_int, ctypes.c_double, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int]
+        lib.oracle_attention_rows.restype = ctypes.c_int
+        lib.oracle_threads.argtypes = []
+        lib.oracle_threads.restype = ctypes.c_int
+        _LIB = lib
+    return _LIB
+
+
+def _bits(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("oracle inputs are bf16 bit patterns (uint16)")
+    return a
+
+
+def default_threads() -> int:
+    return int(_lib().oracle_threads())
+
+
+def attention_fwd(q, k, v, causal: bool, scale: float, threads: int = 0):
+    """O (fp64 [B,H,N,d]) and LSE (fp64 [B,H,N]) for bf16-bit inputs [B,H,N,d]."""
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    B, H, N, d = q.shape
+    assert k.shape == q.shape and v.shape == q.shape
+    o = np.zeros((B, H, N, d), dtype=np.float64)
+    lse = np.zeros((B, H, N), dtype=np.float64)
+    rc = _lib().oracle_attention_fwd(q.ctypes.data, k.ctypes.data, v.ctypes.data, o.ctypes.data,
+                                     lse.ctypes.data, B, H, N, d, int(bool(causal)),
+                                     float(scale), int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_fwd failed ({rc})")
+    return o, lse
+
+
+def attention_rows(q, k, v, causal: bool, scale: float, rows, threads: int = 0):
+    """O and LSE for selected rows only; rows are flat indices bh * N + i."""
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    B, H, N, d = q.shape
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    o = np.zeros((len(r), d), dtype=np.float64)
+    lse = np.zeros(len(r), dtype=np.float64)
+    rc = _lib().oracle_attention_rows(q.ctypes.data, k.ctypes.data, v.ctypes.data, B, H, N, d,
+                                      int(bool(causal)), float(scale), r.ctypes.data, len(r),
+                                      o.ctypes.data, lse.ctypes.data, int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_rows failed ({rc})")
+    return o, lse
