@@ -1,0 +1,12 @@
+"""B200 (sm_100a) fused attention forward: O = softmax(scale * Q K^T [+ causal mask]) V and
+the per-row logsumexp, computed by hand-written tcgen05/TMA kernels behind the C ABI in
+include/fa.h.  This package is the thin Python binding of that library."""
+from ._binding import (FA_ERR_ALIGN, FA_ERR_ARCH, FA_ERR_CUDA, FA_ERR_HEADDIM, FA_ERR_NULL,
+                       FA_ERR_SCALE, FA_ERR_SHAPE, FA_ERR_TIMEOUT, FA_OK, FaError, LIB_PATH,
+                       fa_fwd, fa_fwd_host, header_functions, launches_per_call, lib, strerror,
+                       version)
+
+__all__ = ["fa_fwd", "fa_fwd_host", "FaError", "strerror", "version", "launches_per_call",
+           "header_functions", "lib", "LIB_PATH", "FA_OK", "FA_ERR_NULL", "FA_ERR_SHAPE",
+           "FA_ERR_HEADDIM", "FA_ERR_ALIGN", "FA_ERR_SCALE", "FA_ERR_CUDA", "FA_ERR_TIMEOUT",
+           "FA_ERR_ARCH"]

@@ -1,0 +1,165 @@
+"""ctypes binding of libfa_b200.so (include/fa.h).
+
+Argument marshalling only: every step of the attention forward pass runs in
+the library's CUDA kernels.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the library is missing or the device is not
+sm_100, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+HEADER = os.path.join(ROOT, "include", "fa.h")
+LIB_PATH = os.path.join(HERE, "libfa_b200.so")
+
+FA_OK = 0
+FA_ERR_NULL = -1
+FA_ERR_SHAPE = -2
+FA_ERR_HEADDIM = -3
+FA_ERR_ALIGN = -4
+FA_ERR_SCALE = -5
+FA_ERR_CUDA = -6
+FA_ERR_TIMEOUT = -7
+FA_ERR_ARCH = -8
+
+_i64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str = "fa_fwd"):
+        self.status = status
+        super().__init__(f"{where} failed with status {status}: {strerror(status)}")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python -m attention_forward_17_b200.build` "
+            "(there is no non-CUDA fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.fa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.c_int,
+                           ctypes.c_float, _vp]
+    lib.fa_fwd.restype = ctypes.c_int
+    lib.fa_fwd_status.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.c_int,
+                                  ctypes.c_float, _vp, _vp]
+    lib.fa_fwd_status.restype = ctypes.c_int
+    lib.fa_fwd_host.argtypes = [_vp] * 10 + [_i64, _i64, _i64, _i64, ctypes.c_int, ctypes.c_float,
+                                            _vp]
+    lib.fa_fwd_host.restype = ctypes.c_int
+    lib.fa_fwd_launches.argtypes = [_i64, _i64, _i64, _i64]
+    lib.fa_fwd_launches.restype = ctypes.c_int
+    lib.fa_strerror.argtypes = [ctypes.c_int]
+    lib.fa_strerror.restype = ctypes.c_char_p
+    lib.fa_version.argtypes = []
+    lib.fa_version.restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/fa.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fa_\w+)\s*\(", text, flags=re.M)
+
+
+def strerror(status: int) -> str:
+    return lib.fa_strerror(int(status)).decode()
+
+
+def version() -> tuple[int, int]:
+    v = lib.fa_version()
+    return v >> 16, v & 0xFFFF
+
+
+def launches_per_call(B: int, H: int, N: int, d: int) -> int:
+    return int(lib.fa_fwd_launches(B, H, N, d))
+
+
+def _check_qkv(q, k, v):
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [B, H, N, d], got shape {tuple(t.shape)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError(f"q, k, v shapes differ: {tuple(q.shape)} {tuple(k.shape)} {tuple(v.shape)}")
+    if not (q.device == k.device == v.device) or q.device.type != "cuda":
+        raise ValueError("q, k, v must be on the same CUDA device")
+
+
+def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+           stream=None, status=None):
+    """O, LSE = attention forward of bf16 [B, H, N, d] CUDA tensors.
+
+    ``out`` (bf16 [B,H,N,d]) and ``lse`` (fp32 [B,H,N]) are allocated when not
+    given.  Runs on ``stream`` (a torch.cuda.Stream) or the current stream.
+    ``status`` may be an int32 CUDA tensor with one element; it then receives
+    FA_ERR_TIMEOUT should a device-side wait run out of time.
+    """
+    import torch
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if out.dtype != torch.bfloat16 or out.shape != q.shape or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
+    s = (stream if stream is not None else torch.cuda.current_stream(q.device)).cuda_stream
+    with torch.cuda.device(q.device):
+        if status is None:
+            rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                            lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale), s)
+        else:
+            rc = lib.fa_fwd_status(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                   status.data_ptr(), s)
+    if rc != FA_OK:
+        raise FaError(rc)
+    return out, lse
+
+
+def fa_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal: bool = False,
+                scale: float | None = None, stream=None):
+    """Host-to-host attention forward through caller-provided device buffers.
+
+    All arguments are torch tensors: the ``*_h`` ones on the CPU (pinned for
+    asynchronous copies), the ``*_d`` ones on the GPU.  Enqueues H2D copies,
+    the kernel and D2H copies on ``stream`` and returns without waiting.
+    """
+    import torch
+    _check_qkv(q_d, k_d, v_d)
+    B, H, N, d = q_d.shape
+    for t in (q_h, k_h, v_h, o_h):
+        if t.shape != q_d.shape or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("host q/k/v/o must be contiguous bf16 tensors shaped like q_d")
+    if tuple(lse_h.shape) != (B, H, N) or lse_h.dtype != torch.float32:
+        raise ValueError("lse_h must be fp32 [B, H, N]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    s = (stream if stream is not None else torch.cuda.current_stream(q_d.device)).cuda_stream
+    with torch.cuda.device(q_d.device):
+        rc = lib.fa_fwd_host(q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), o_h.data_ptr(),
+                             lse_h.data_ptr(), q_d.data_ptr(), k_d.data_ptr(), v_d.data_ptr(),
+                             o_d.data_ptr(), lse_d.data_ptr(), B, H, N, d, int(bool(causal)),
+                             float(scale), s)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_host")

@@ -1,0 +1,60 @@
+"""Builds libfa_b200.so, the sm_100a attention library, in-tree with nvcc.
+
+The library is self-contained: CUDA runtime linked statically, the driver's
+tensor-map encoder fetched at run time, no torch symbols.
+"""
+from __future__ import annotations
+
+import glob
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+
+NVCC_FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-std=c++17", "-lineinfo",
+    "-Xcompiler", "-fPIC", "-shared",
+    "-Xptxas", "-v",
+]
+
+
+def library_path() -> str:
+    return os.path.join(HERE, "libfa_b200.so")
+
+
+def _sources():
+    return [os.path.join(CSRC, "fa_fwd.cu")]
+
+
+def _deps():
+    return (glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+            + glob.glob(os.path.join(ROOT, "include", "*.h")))
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    out = library_path()
+    if (not force and os.path.exists(out)
+            and all(os.path.getmtime(out) >= os.path.getmtime(p) for p in _deps())):
+        return out
+    nvcc = os.environ.get("NVCC", "nvcc")
+    tmp = out + ".tmp"
+    cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), *_sources(), "-o", tmp]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    log = res.stdout + res.stderr
+    with open(os.path.join(HERE, "build.log"), "w") as f:
+        f.write(" ".join(cmd) + "\n" + log)
+    if res.returncode != 0:
+        sys.stderr.write(log)
+        raise RuntimeError("nvcc failed building libfa_b200.so")
+    if verbose:
+        sys.stdout.write(log)
+    os.replace(tmp, out)
+    return out
+
+
+if __name__ == "__main__":
+    print(build(force=True, verbose=True))

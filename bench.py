@@ -1,0 +1,403 @@
+#!/usr/bin/env python3
+"""Benchmark of the sm_100a fused attention forward pass.
+
+One step = one forward pass of the workload in BOTH masking modes (the
+non-causal and the causal call, inputs resident in HBM).  Rank 0 prints one
+JSON line:
+
+  value        whole-job TFLOP/s (4*B*H*N^2*d non-causal + 2*B*H*N^2*d causal per
+               step, summed over ranks, divided by the max over ranks of the
+               device-timed region)
+  e2e          the same metric through the host-buffer entry point (pinned host
+               Q/K/V copied in, O/LSE copied out, inside the timed region)
+  roofline     the attention kernel against the measured dense bf16 peak
+  cpu_baseline the fp64 oracle on the host cores, on a bounded sample of rows
+
+`--impl reference` times the fp64 oracle instead (the reference arm of this
+build: there is no other implementation of the pages to run).
+
+Multi-GPU (`torchrun --nproc-per-node N bench.py --gpus N`): the work is
+independent (batch, head) slices, so every rank runs its own replica of the
+workload with no data-path collective (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s (causal/non-causal) and % of B200 dense BF16 peak"
+DATASHEET_BF16_TFLOPS = 2250.0
+
+WORKLOADS = {
+    # the headline workload: N >= 4096, d = 128, both masking modes, wide score range
+    "b1_h32_n16384_d128_qk_sigma3": dict(B=1, H=32, N=16384, d=128, sigma_qk=3.0),
+    "b2_h16_n4096_d128": dict(B=2, H=16, N=4096, d=128, sigma_qk=1.0),
+    "b4_h8_n1024_d64": dict(B=4, H=8, N=1024, d=64, sigma_qk=1.0),
+}
+DEFAULT_WORKLOAD = "b1_h32_n16384_d128_qk_sigma3"
+
+
+def flops(B, H, N, d, causal):
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(bf16=float(p["bf16_tflops"]), bf16_sustained=float(p["bf16_tflops_sustained"]),
+                    hbm=float(p["hbm_gbs"]), source="measured")
+    except Exception:
+        return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu_index), "-lms", "100"], stdout=self.out,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 active=parts[4], hw=parts[5], hwt=parts[6], swt=parts[7],
+                                 pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [r for r in rows if r["power"] > 300] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["smax"] for r in rows),
+                "power_w_max": max(r["power"] for r in rows),
+                "samples": len(load), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def oracle_sample(bits, cfg, target_s, seed=0):
+    """Time the fp64 oracle on a bounded sample of rows of the workload, both
+    modes; returns (TFLOP/s by the metric's per-row FLOP convention, details)."""
+    import numpy as np
+    import oracle
+    q, k, v = bits
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d)
+    rng = np.random.default_rng(seed)
+    threads = oracle.default_threads()
+    nrows, spent, done_flops, results = 8, 0.0, 0.0, []
+    while True:
+        rows = np.sort(rng.choice(B * H * N, nrows, replace=False)).astype(np.int64)
+        step_flops, t0 = 0.0, time.perf_counter()
+        outs = {}
+        for causal in (False, True):
+            outs[causal] = oracle.attention_rows(q, k, v, causal, scale, rows)
+            # per-row share of the metric's FLOP convention
+            step_flops += nrows * (4.0 * N * d / (2 if causal else 1))
+        dt = time.perf_counter() - t0
+        spent += dt
+        done_flops += step_flops
+        results.append((rows, outs))
+        if spent >= target_s or nrows >= B * H * N // 4:
+            break
+        nrows = min(B * H * N // 4, max(nrows * 2, int(nrows * target_s / max(dt, 1e-3) * 0.5)))
+    return done_flops / spent / 1e12, dict(seconds=spent, cores=threads, results=results,
+                                           rows=sum(len(r[0]) for r in results))
+
+
+def sample_parity(results, o_by_mode, lse_by_mode, d):
+    import numpy as np
+    worst = dict(o_max_abs=0.0, lse_max_abs=0.0)
+    for rows, outs in results:
+        for causal, (o_ref, lse_ref) in outs.items():
+            o = o_by_mode[causal].view(-1, d)[rows].float().cpu().numpy().astype(np.float64)
+            lse = lse_by_mode[causal].view(-1)[rows].cpu().numpy().astype(np.float64)
+            worst["o_max_abs"] = max(worst["o_max_abs"], float(np.abs(o - o_ref).max()))
+            worst["lse_max_abs"] = max(worst["lse_max_abs"], float(np.abs(lse - lse_ref).max()))
+    worst["pass"] = worst["o_max_abs"] <= 2e-2 and worst["lse_max_abs"] <= 1e-3
+    return worst
+
+
+# ------------------------------------------------------------------ arms
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    return world, rank, local
+
+
+def run_reference(args, cfg):
+    """The oracle arm: fp64 CPU attention on bounded row samples per step."""
+    world, rank, _ = dist_setup(args.gpus)
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    import seeded_inputs as si
+    B, H, N, d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
+    bits = si.make_qkv(B, H, N, d, seed=0, sigma_qk=cfg["sigma_qk"])
+    q, k, v = bits
+    scale = 1.0 / math.sqrt(d)
+    rows_per_step = max(8, args.ref_rows)
+    rng = np.random.default_rng(0)
+
+    def step():
+        rows = np.sort(rng.choice(B * H * N, rows_per_step, replace=False)).astype(np.int64)
+        f = 0.0
+        for causal in (False, True):
+            oracle.attention_rows(q, k, v, causal, scale, rows)
+            f += rows_per_step * 4.0 * N * d / (2 if causal else 1)
+        return f
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    total = sum(step() for _ in range(args.steps))
+    dt = time.perf_counter() - t0
+    value = total / dt / 1e12
+    sample = (f"{rows_per_step} random query rows per step, each in both masking modes, of "
+              f"B={B},H={H},N={N},d={d}; complete fp64 score rows")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args.workload, cfg, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.default_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(name, cfg, n_gpus):
+    return {"workload": name, "B": cfg["B"], "H": cfg["H"], "N": cfg["N"], "d": cfg["d"],
+            "qk_sigma": cfg["sigma_qk"], "v_sigma": 1.0, "scale": "1/sqrt(d)",
+            "modes": ["non-causal", "causal"], "seed": 0,
+            "l2": "inputs (Q,K,V = 3 x {:.0f} MiB) larger than the 126 MB L2".format(
+                cfg["B"] * cfg["H"] * cfg["N"] * cfg["d"] * 2 / 2 ** 20),
+            "parallelism": f"replicas x{n_gpus} (independent (b,h) slices, no collective)"}
+
+
+def run_ours(args, cfg):
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    import numpy as np
+    import attention_forward_17_b200 as fa
+    import seeded_inputs as si
+
+    B, H, N, d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
+    bits = si.make_qkv(B, H, N, d, seed=rank, sigma_qk=cfg["sigma_qk"])
+
+    def dev_tensor(b):
+        return torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v = (dev_tensor(b) for b in bits)
+    o = {c: torch.empty_like(q) for c in (False, True)}
+    lse = {c: torch.empty((B, H, N), dtype=torch.float32, device=dev) for c in (False, True)}
+    stream = torch.cuda.current_stream(dev)
+    f_step = flops(B, H, N, d, False) + flops(B, H, N, d, True)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------- device-resident timing, per-launch events
+    for _ in range(args.warmup):
+        for c in (False, True):
+            fa.fa_fwd(q, k, v, causal=c, out=o[c], lse=lse[c])
+    torch.cuda.synchronize()
+    ev = {c: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)] for c in (False, True)}
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gpu_index = local
+    with ClockSampler(gpu_index) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for s in range(args.steps):
+            for c in (False, True):
+                ev[c][s][0].record(stream)
+                fa.fa_fwd(q, k, v, causal=c, out=o[c], lse=lse[c])
+                ev[c][s][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    launch_ms = {c: statistics.mean(a.elapsed_time(b) for a, b in ev[c]) for c in (False, True)}
+    clocks = clk.summary()
+    value = world * f_step * args.steps / (elapsed_ms / 1e3) / 1e12
+
+    # ---------------- end to end through the host-buffer entry point
+    e2e = None
+    if not args.no_e2e:
+        host = [torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).pin_memory() for b in bits]
+        o_h = {c: torch.empty_like(host[0]).pin_memory() for c in (False, True)}
+        l_h = {c: torch.empty((B, H, N), dtype=torch.float32).pin_memory() for c in (False, True)}
+        qd, kd, vd = (torch.empty_like(q) for _ in range(3))
+        e2e_steps = max(1, min(args.steps, 10))
+
+        def e2e_step():
+            for c in (False, True):
+                fa.fa_fwd_host(host[0], host[1], host[2], o_h[c], l_h[c], qd, kd, vd, o[c], lse[c],
+                               causal=c)
+
+        for _ in range(max(1, min(args.warmup, 3))):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(a.elapsed_time(b))
+        tensor_bytes = B * H * N * d * 2
+        e2e = {"value": world * f_step * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 2 * 3 * tensor_bytes,
+               "d2h_bytes_per_step": 2 * (tensor_bytes + B * H * N * 4),
+               "steps": e2e_steps, "entry_point": "fa_fwd_host"}
+
+    # ---------------- roofline of the dominant launch (non-causal instantiation)
+    peaks = load_peaks()
+    ach = {c: flops(B, H, N, d, c) / (launch_ms[c] / 1e3) / 1e12 for c in (False, True)}
+    dominant = False if launch_ms[False] >= launch_ms[True] else True
+    roofline = {"bound": "tensor", "kernel": f"fa_fwd_kernel<{d},{str(dominant).lower()}>",
+                "achieved": ach[dominant], "peak": peaks["bf16"], "unit": "TFLOP/s",
+                "frac": ach[dominant] / peaks["bf16"], "peak_source": peaks["source"] + " burst",
+                "traffic": None,
+                "per_mode": {("causal" if c else "non_causal"): {
+                    "ms_per_launch": launch_ms[c], "tflops": ach[c],
+                    "frac_of_measured_burst": ach[c] / peaks["bf16"],
+                    "frac_of_measured_sustained": ach[c] / peaks["bf16_sustained"],
+                    "frac_of_datasheet_2250": ach[c] / DATASHEET_BF16_TFLOPS} for c in (False, True)}}
+
+    # ---------------- CPU baseline (rank 0, N=1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_cpu, det = oracle_sample(bits, cfg, args.cpu_seconds)
+        par = sample_parity(det["results"], o, lse, d)
+        cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": det["cores"], "kind": "oracle",
+               "sample": f"{det['rows']} random query rows of the workload, each in both masking "
+                         f"modes (complete fp64 score rows), {det['seconds']:.1f} s",
+               "sample_parity_vs_gpu": par}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": workload_config(args.workload, cfg, world),
+            "pct_of_peak": {"measured_burst": 100 * value / world / peaks["bf16"],
+                            "measured_sustained": 100 * value / world / peaks["bf16_sustained"],
+                            "datasheet_2250": 100 * value / world / DATASHEET_BF16_TFLOPS},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps * 2 * fa.launches_per_call(B, H, N, d),
+            "clocks": clocks, "impl": "ours",
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle sample")
+    ap.add_argument("--ref-rows", type=int, default=64,
+                    help="query rows per step of the reference (oracle) arm")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    cfg = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

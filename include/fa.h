@@ -1,0 +1,120 @@
+/*
+ * fa.h - C ABI of the B200 (sm_100a) fused attention forward library
+ * (libfa_b200.so).
+ *
+ * The operation is the fused FlashAttention forward pass of the "TileLang
+ * tutorial" (FlashAttention section): query, key and value tiles are processed
+ * without materialising the attention-score matrix in global memory, using an
+ * online softmax (running row maxima, running normalisation sums, rescaling
+ * factors) and tensor-core products, for causal and non-causal attention.  For
+ * every (b, h) slice and query row i it returns
+ *
+ *     O[b,h,i,:] = sum_j softmax_j( scale * Q[b,h,i,:] . K[b,h,j,:] ) * V[b,h,j,:]
+ *     LSE[b,h,i] = ln sum_j exp( scale * Q[b,h,i,:] . K[b,h,j,:] )
+ *
+ * where, when `causal` is nonzero, only keys j <= i take part (top-left
+ * alignment; query and key lengths are equal).  The pages validate this
+ * against scaled-dot-product attention; LSE is the natural-log logsumexp of the
+ * scaled scores.
+ *
+ * Layout: Q, K, V and O are bf16 [B, H, N, d], dense row-major (d fastest), in
+ * device memory.  LSE is fp32 [B, H, N].  d must be 64 or 128.  Arithmetic:
+ * bf16 tensor-core products with fp32 accumulation, fp32 softmax, P rounded to
+ * bf16 (nearest-even) before the P.V product, O rounded to bf16 (nearest-even).
+ *
+ * Ownership: the caller owns every buffer.  The library never allocates device
+ * memory and keeps no per-call state.
+ *
+ * Errors: the argument checks below run on the host in the listed order and
+ * return before anything is launched.  Launches are asynchronous on `stream`
+ * (a cudaStream_t; NULL = the legacy default stream); a launch failure returns
+ * FA_ERR_CUDA.  The calls never synchronise the stream.
+ *
+ * Threading: every entry point is reentrant and may be called from several
+ * host threads at once.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_NULL = -1,     /* a required pointer is NULL                              */
+    FA_ERR_SHAPE = -2,    /* B, H or N negative, or beyond the supported range       */
+    FA_ERR_HEADDIM = -3,  /* d is not 64 or 128                                      */
+    FA_ERR_ALIGN = -4,    /* a device pointer is not 16-byte aligned (LSE: 4-byte)   */
+    FA_ERR_SCALE = -5,    /* scale is not finite and > 0                             */
+    FA_ERR_CUDA = -6,     /* a CUDA runtime/driver call failed                       */
+    FA_ERR_TIMEOUT = -7,  /* a device-side pipeline wait ran out of time             */
+    FA_ERR_ARCH = -8      /* the current device is not compute capability 10.0       */
+} fa_status;
+
+/*
+ * fa_fwd - fused attention forward.
+ *
+ *   q, k, v  device, bf16 [B,H,N,d], read only, 16-byte aligned.
+ *   o        device, bf16 [B,H,N,d], written, 16-byte aligned.
+ *   lse      device, fp32 [B,H,N], written, 4-byte aligned.
+ *   B, H, N  >= 0; a zero makes the call a no-op that returns FA_OK (pointers
+ *            are then not examined).  N <= 2^31 - 512 and B*H <= 2^31 - 1.
+ *   d        64 or 128.
+ *   causal   0 = full attention, nonzero = key j visible to query i iff j <= i.
+ *   scale    multiplier of q.k inside the softmax (usually 1/sqrt(d)); finite, > 0.
+ *   stream   cudaStream_t or NULL.
+ *
+ * o and lse must not overlap q, k or v (not checked).  Should a device-side
+ * pipeline wait ever exceed about two seconds (it cannot in correct
+ * operation), the affected query rows receive LSE = NaN and the kernel still
+ * terminates; use fa_fwd_status to also receive FA_ERR_TIMEOUT in a status
+ * word.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+           int64_t N, int64_t d, int causal, float scale, void* stream);
+
+/*
+ * fa_fwd_status - fa_fwd that also reports device-side failures.
+ *
+ *   dev_status  device int, caller-owned.  The kernel never clears it; it
+ *               writes FA_ERR_TIMEOUT into it if a pipeline wait runs out of
+ *               time.  Read it after the stream has completed.  NULL behaves
+ *               like fa_fwd.
+ * Other arguments and checks are those of fa_fwd.
+ */
+int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                  int64_t H, int64_t N, int64_t d, int causal, float scale, int* dev_status,
+                  void* stream);
+
+/*
+ * fa_fwd_host - the same computation starting from and ending in host memory.
+ *
+ * Enqueues on `stream`: copies q_h, k_h, v_h (host, bf16 [B,H,N,d]; pinned
+ * memory makes the copies asynchronous) into the caller's device buffers q_d,
+ * k_d, v_d; runs fa_fwd on them into o_d and lse_d; copies o_d and lse_d back
+ * into o_h and lse_h (host).  Nothing is allocated; the call returns without
+ * synchronising, so the host buffers must stay valid until the stream has
+ * completed.  Argument checks are those of fa_fwd applied to the device
+ * buffers, plus FA_ERR_NULL for a NULL host pointer.
+ */
+int fa_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, float* lse_h,
+                void* q_d, void* k_d, void* v_d, void* o_d, float* lse_d, int64_t B, int64_t H,
+                int64_t N, int64_t d, int causal, float scale, void* stream);
+
+/* Number of kernel launches one fa_fwd call makes for these sizes (0 or 1). */
+int fa_fwd_launches(int64_t B, int64_t H, int64_t N, int64_t d);
+
+/* Static description of a status code; never NULL. */
+const char* fa_strerror(int status);
+
+/* Library ABI version, (major << 16) | minor. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

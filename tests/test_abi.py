@@ -1,0 +1,101 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function
+include/fa.h declares, and rejects bad arguments on the host, in the
+documented order, before touching the device."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import attention_forward_17_b200 as fa
+from attention_forward_17_b200 import _binding as bnd
+
+LIB = fa.lib
+
+
+def test_exports_every_header_function():
+    names = fa.header_functions()
+    assert set(names) >= {"fa_fwd", "fa_fwd_status", "fa_fwd_host", "fa_strerror", "fa_version",
+                          "fa_fwd_launches"}
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, f"{n} declared in include/fa.h but not exported"
+        assert hasattr(LIB, n)
+
+
+def test_no_torch_in_library():
+    out = subprocess.run(["ldd", fa.LIB_PATH], capture_output=True, text=True).stdout
+    assert "torch" not in out and "c10" not in out
+
+
+def test_strerror_and_version():
+    for code in range(-8, 1):
+        s = fa.strerror(code)
+        assert isinstance(s, str) and s
+    assert fa.strerror(12345) == "unknown status"
+    assert fa.version() == (1, 0)
+
+
+def call(q=16, k=32, v=48, o=64, lse=80, B=1, H=1, N=128, d=64, causal=0, scale=0.125):
+    # fake, never-dereferenced device addresses: every case below fails a host check first
+    return LIB.fa_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), fa.FA_ERR_SHAPE),
+    (dict(N=-5), fa.FA_ERR_SHAPE),
+    (dict(q=0), fa.FA_ERR_NULL),
+    (dict(lse=0), fa.FA_ERR_NULL),
+    (dict(N=2 ** 31), fa.FA_ERR_SHAPE),
+    (dict(B=2 ** 20, H=2 ** 12), fa.FA_ERR_SHAPE),
+    (dict(d=96), fa.FA_ERR_HEADDIM),
+    (dict(d=256), fa.FA_ERR_HEADDIM),
+    (dict(q=18), fa.FA_ERR_ALIGN),
+    (dict(o=72), fa.FA_ERR_ALIGN),
+    (dict(lse=82), fa.FA_ERR_ALIGN),
+    (dict(scale=0.0), fa.FA_ERR_SCALE),
+    (dict(scale=-1.0), fa.FA_ERR_SCALE),
+    (dict(scale=float("inf")), fa.FA_ERR_SCALE),
+    (dict(scale=float("nan")), fa.FA_ERR_SCALE),
+])
+def test_argument_errors(kw, code):
+    assert call(**kw) == code
+
+
+def test_error_order():
+    # shape before null before head-dim before alignment before scale
+    assert call(B=-1, q=0) == fa.FA_ERR_SHAPE
+    assert call(q=0, d=96) == fa.FA_ERR_NULL
+    assert call(d=96, q=18) == fa.FA_ERR_HEADDIM
+    assert call(q=18, scale=0.0) == fa.FA_ERR_ALIGN
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(H=0), dict(N=0)])
+def test_empty_problem_is_a_noop(kw):
+    # pointers are not examined for an empty problem
+    assert call(q=0, k=0, v=0, o=0, lse=0, d=96, **kw) == fa.FA_OK
+
+
+def test_host_entry_checks():
+    f = LIB.fa_fwd_host
+    args = [1024, 2048, 3072, 4096, 5120, 16, 32, 48, 64, 80]
+    bad = list(args)
+    bad[0] = 0
+    assert f(*bad, 1, 1, 128, 64, 0, 0.125, None) == fa.FA_ERR_NULL
+    bad = list(args)
+    bad[5] = 18
+    assert f(*bad, 1, 1, 128, 64, 0, 0.125, None) == fa.FA_ERR_ALIGN
+    assert f(*args, 1, 1, 0, 64, 0, 0.125, None) == fa.FA_OK
+
+
+def test_launch_count():
+    assert fa.launches_per_call(1, 1, 128, 64) == 1
+    assert fa.launches_per_call(0, 1, 128, 64) == 0
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(bnd, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        bnd._load()
