@@ -21,7 +21,10 @@
 //               only when m grows by more than 2^8 (lazy rescale; the final
 //               O / l uses the same stale m, so it is exact), write P_t as
 //               bf16 into TMEM over S_t, and finally normalise and store O_t
-//               and LSE.
+//               and LSE.  O is divided by the sum of the bf16-rounded weights
+//               the P V product actually used, so every O row is an exact
+//               convex combination of V rows (a one-hot row returns its V row
+//               unchanged); LSE uses the fp32 sum of the unrounded weights.
 //
 // TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
 // O_1 [256+D, 256+2D).  P_t (bf16, two per column) sits in the upper half of
@@ -191,7 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float c = p.scale_log2;
 
         float m_run = -INFINITY;   // running max of scale*log2(e)*s (possibly stale by < 8)
-        float l_run = 0.f;         // running sum of 2^(c*s - m_run)
+        float l_run = 0.f;         // running sum of 2^(c*s - m_run), fp32 (for LSE)
+        float lh_run = 0.f;        // running sum of the same weights rounded to bf16 (for O)
 
         for (int j = 0; j < n_kv; ++j) {
             wait_bar(bar_s_full + 8 * t, j & 1, abort, p.status);
@@ -228,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 alpha = ex2_approx(m_run - m_new);
                 m_run = m_new;
                 l_run *= alpha;
+                lh_run *= alpha;
             }
             if (j > 0 && __any_sync(0xffffffffu, grow)) {
                 // O_t holds sum_{j' < j} P V with the old reference max: scale
@@ -245,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-            float sum0 = 0.f, sum1 = 0.f;
+            float sum0 = 0.f, sum1 = 0.f, sumh0 = 0.f, sumh1 = 0.f;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[32];
@@ -258,11 +263,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float p1 = ex2_approx(fmaf(x1, c, -m_use));
                     sum0 += p0;
                     sum1 += p1;
-                    pk[i] = pack_bf16x2(p0, p1);
+                    const uint32_t w = pack_bf16x2(p0, p1);
+                    sumh0 += __uint_as_float(w << 16);
+                    sumh1 += __uint_as_float(w & 0xffff0000u);
+                    pk[i] = w;
                 }
                 tmem_st32(t_p + 32 * h, pk);
             }
             l_run += sum0 + sum1;
+            lh_run += sumh0 + sumh1;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p_full + 8 * t);
@@ -272,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         wait_bar(bar_o_full + 8 * t, 0, abort, p.status);
         tc_fence_after();
         const bool valid = row < p.N;
-        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+        const float inv_l = lh_run > 0.f ? 1.f / lh_run : 0.f;
         __nv_bfloat16* orow = p.o + (static_cast<int64_t>(bh) * p.N + row) * D;
 #pragma unroll 1
         for (int q = 0; q < D / 32; ++q) {
