@@ -25,11 +25,20 @@ DeviceState g_devices[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
+// Opts the instantiation into its dynamic shared memory and checks that it was
+// compiled with enough registers for the in-kernel warpgroup rebalance (a
+// setmaxnreg.inc asking for more than the launch allocated would never
+// return).
 template <int D, bool CAUSAL>
-cudaError_t set_smem_attr() {
-    return cudaFuncSetAttribute(fa::fa_fwd_kernel<D, CAUSAL>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                fa::TileCfg<D>::kSmemBytes);
+int set_smem_attr() {
+    if (cudaFuncSetAttribute(fa::fa_fwd_kernel<D, CAUSAL>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::TileCfg<D>::kSmemBytes) != cudaSuccess)
+        return FA_ERR_CUDA;
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, fa::fa_fwd_kernel<D, CAUSAL>) != cudaSuccess) return FA_ERR_CUDA;
+    if (attr.numRegs * fa::kThreads < fa::kRegSplitTotal) return FA_ERR_CUDA;
+    return FA_OK;
 }
 
 // One-time per-device set-up: architecture check and the shared-memory opt-in
@@ -40,9 +49,10 @@ int device_setup(int dev) {
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
         return FA_ERR_CUDA;
     if (major != 10 || minor != 0) return FA_ERR_ARCH;
-    if (set_smem_attr<64, false>() != cudaSuccess || set_smem_attr<64, true>() != cudaSuccess ||
-        set_smem_attr<128, false>() != cudaSuccess || set_smem_attr<128, true>() != cudaSuccess)
-        return FA_ERR_CUDA;
+    int rc;
+    if ((rc = set_smem_attr<64, false>()) != FA_OK || (rc = set_smem_attr<64, true>()) != FA_OK ||
+        (rc = set_smem_attr<128, false>()) != FA_OK || (rc = set_smem_attr<128, true>()) != FA_OK)
+        return rc;
     return FA_OK;
 }
 

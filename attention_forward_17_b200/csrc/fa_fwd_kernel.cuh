@@ -10,7 +10,8 @@
 // FlashAttention section).
 //
 // Blackwell mapping (one CTA = 256 query rows of one (b, h) slice, as two
-// 128-row tiles t = 0, 1 processed in ping-pong):
+// 128-row tiles t = 0, 1 processed in ping-pong; 384 threads, and the
+// softmax warpgroups take registers from the third warpgroup with setmaxnreg):
 //   warp 8      TMA producer: Q tiles once, then K_j / V_j tiles through a
 //               ring of shared-memory slots (mbarrier full/empty pairs).
 //   warp 9      MMA issuer (one thread): S_t = Q_t K_j^T into tensor memory
@@ -44,13 +45,20 @@
 
 namespace fa {
 
-constexpr int kThreads = 320;     // 8 softmax warps + producer warp + MMA warp
+constexpr int kThreads = 384;     // 2 softmax warpgroups + 1 warpgroup (producer, MMA, 2 spare)
 constexpr int kBlockM = 128;      // query rows per tile (= TMEM lanes)
 constexpr int kBlockN = 128;      // key rows per tile
 constexpr int kTilesPerCta = 2;   // ping-pong query tiles
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kStatusTimeout = -7;  // FA_ERR_TIMEOUT
+// Per-thread registers after the warpgroups rebalance (launch: 384 x 168).
+constexpr uint32_t kRegsSoftmax = 208;
+constexpr uint32_t kRegsOther = 88;
+constexpr int kRegSplitTotal = 2 * 128 * kRegsSoftmax + 128 * kRegsOther;  // 64512 = 384 x 168
+// Every kEmuEvery-th pair of exponentials is evaluated on the FMA pipe by
+// polynomial instead of on the special-function unit (0 = never).
+constexpr int kEmuEvery = 4;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;      // 2 s
 constexpr uint64_t kWaitLimitAbortNs = 1000000ull;    // 1 ms once the CTA has aborted
 
@@ -95,7 +103,7 @@ struct FwdParams {
 };
 
 // ---------------------------------------------------------------- bounded waits
-__device__ __noinline__ void wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
+__device__ __forceinline__ void wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
                                        int* status) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
@@ -116,6 +124,38 @@ __device__ __noinline__ void wait_slow(uint32_t bar, uint32_t parity, volatile u
 __device__ __forceinline__ void wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
                                          int* status) {
     if (!mbar_try_wait(bar, parity)) wait_slow(bar, parity, abort, status);
+}
+
+// ---------------------------------------------------------------- exp2 on the FMA pipe
+// 2^x for two values without the special-function unit (Cody-Waite style
+// split x = j + f):
+//   j = floor(x): add 1.5 * 2^23 rounding toward -inf, so the sum's low
+//       mantissa bits hold j; subtract the constant back (exact);
+//   f = x - j in [0, 1) (exact);
+//   2^f ~ 1 + f (a1 + f (a2 + f a3)), a degree-3 minimax fit in relative
+//       error with p(0) = 1 (fit_exp2_poly.py: max relative error 8.6e-5);
+//   2^j is applied by adding j << 23 to the bits of 2^f (the low bits of the
+//       rounded sum shifted into the exponent field).
+// x is clamped to >= -126 so the result stays a normal float (and -inf maps
+// to 2^-126, which vanishes next to the row maximum's weight >= 1).
+constexpr float kExp2A1 = 0.6951167583465576f;
+constexpr float kExp2A2 = 0.22764499485492706f;
+constexpr float kExp2A3 = 0.07706703990697861f;
+
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    const uint64_t x = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const uint64_t t = add2_rm(x, f2(kMagic, kMagic));
+    const uint64_t jf = add2(t, f2(-kMagic, -kMagic));
+    const uint64_t fr = fma2(jf, f2(-1.f, -1.f), x);
+    uint64_t q = fma2(f2(kExp2A3, kExp2A3), fr, f2(kExp2A2, kExp2A2));
+    q = fma2(q, fr, f2(kExp2A1, kExp2A1));
+    q = fma2(q, fr, f2(1.f, 1.f));
+    float q0, q1, t0, t1;
+    f2_split(q, q0, q1);
+    f2_split(t, t0, t1);
+    y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -182,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = bars->tmem_base;
 
     if (warp < 8) {
+        regs_increase<kRegsSoftmax>();
         // ============================================================ softmax
         const int t = warp >> 2;                  // query tile of this warpgroup
         const int r = threadIdx.x & 127;          // row within the tile = TMEM lane
@@ -197,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float l_run = 0.f;         // running sum of 2^(c*s - m_run), fp32 (for LSE)
         float lh_run = 0.f;        // running sum of the same weights rounded to bf16 (for O)
 
+        const uint64_t c2 = f2(c, c);
         for (int j = 0; j < n_kv; ++j) {
             wait_bar(bar_s_full + 8 * t, j & 1, abort, p.status);
             tc_fence_after();
@@ -217,15 +259,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 32; ++i)
                         if (32 * q + i >= lim) s[q][i] = __float_as_uint(-INFINITY);
             }
-            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+            // row max: eight independent 3-input max chains
+            float mx[8];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                mx0 = fmaxf(mx0, __uint_as_float(s[0][i]));
-                mx1 = fmaxf(mx1, __uint_as_float(s[1][i]));
-                mx2 = fmaxf(mx2, __uint_as_float(s[2][i]));
-                mx3 = fmaxf(mx3, __uint_as_float(s[3][i]));
+            for (int a = 0; a < 8; ++a) mx[a] = __uint_as_float(s[a >> 1][(a & 1) * 16]);
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                const int q = a >> 1, b0 = (a & 1) * 16;
+#pragma unroll
+                for (int i = 1; i < 15; i += 2)
+                    mx[a] = max3f(mx[a], __uint_as_float(s[q][b0 + i]), __uint_as_float(s[q][b0 + i + 1]));
+                mx[a] = fmaxf(mx[a], __uint_as_float(s[q][b0 + 15]));
             }
-            const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c;
+            const float m_new =
+                max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c;
             const bool grow = m_new > m_run + 8.0f;
             float alpha = 1.f;
             if (grow) {
@@ -250,28 +297,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-            float sum0 = 0.f, sum1 = 0.f, sumh0 = 0.f, sumh1 = 0.f;
+            const uint64_t negm2 = f2(-m_use, -m_use);
+            // p = 2^(c*s - m): pairs of columns through packed FMAs; sums of the
+            // fp32 weights (l, for LSE) and of their bf16 roundings (for O)
+            uint64_t l2a = 0, l2b = 0, h2a = 0, h2b = 0;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int col = 64 * h + 2 * i;
-                    const float x0 = __uint_as_float(s[col >> 5][col & 31]);
-                    const float x1 = __uint_as_float(s[(col + 1) >> 5][(col + 1) & 31]);
-                    const float p0 = ex2_approx(fmaf(x0, c, -m_use));
-                    const float p1 = ex2_approx(fmaf(x1, c, -m_use));
-                    sum0 += p0;
-                    sum1 += p1;
+                    const uint64_t x2 = fma2(f2(__uint_as_float(s[col >> 5][col & 31]),
+                                                __uint_as_float(s[col >> 5][(col & 31) + 1])),
+                                             c2, negm2);
+                    float x0, x1;
+                    f2_split(x2, x0, x1);
+                    float p0, p1;
+                    if (kEmuEvery > 0 && (i % kEmuEvery) == kEmuEvery - 1) {
+                        exp2_poly2(x0, x1, p0, p1);
+                    } else {
+                        p0 = ex2_approx(x0);
+                        p1 = ex2_approx(x1);
+                    }
                     const uint32_t w = pack_bf16x2(p0, p1);
-                    sumh0 += __uint_as_float(w << 16);
-                    sumh1 += __uint_as_float(w & 0xffff0000u);
+                    const uint64_t pr = f2(p0, p1);
+                    const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+                    if (i & 1) {
+                        l2b = add2(l2b, pr);
+                        h2b = add2(h2b, ph);
+                    } else {
+                        l2a = add2(l2a, pr);
+                        h2a = add2(h2a, ph);
+                    }
                     pk[i] = w;
                 }
                 tmem_st32(t_p + 32 * h, pk);
             }
-            l_run += sum0 + sum1;
-            lh_run += sumh0 + sumh1;
+            float la0, la1, lb0, lb1, ha0, ha1, hb0, hb1;
+            f2_split(l2a, la0, la1);
+            f2_split(l2b, lb0, lb1);
+            f2_split(h2a, ha0, ha1);
+            f2_split(h2b, hb0, hb1);
+            l_run += (la0 + la1) + (lb0 + lb1);
+            lh_run += (ha0 + ha1) + (hb0 + hb1);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p_full + 8 * t);
@@ -308,6 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             p.lse[static_cast<int64_t>(bh) * p.N + row] = lse;
         }
     } else if (warp == kProducerWarp) {
+        regs_decrease<kRegsOther>();
         // ============================================================ TMA producer
         if (lane == 0) {
             const uint64_t pol_q = policy_evict_first();
@@ -347,7 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-    } else {
+    } else if (warp == kMmaWarp) {
+        regs_decrease<kRegsOther>();
         // ============================================================ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false);
@@ -420,6 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             wait_bar(bar_mma_done, 0, abort, p.status);
         }
         __syncwarp();
+    } else {
+        regs_decrease<kRegsOther>();   // spare warps of the third warpgroup
     }
 
     tc_fence_before();

@@ -43,7 +43,10 @@ WORKLOADS = {
     "b1_h32_n16384_d128_qk_sigma3": dict(B=1, H=32, N=16384, d=128, sigma_qk=3.0),
     "b2_h16_n4096_d128": dict(B=2, H=16, N=4096, d=128, sigma_qk=1.0),
     "b4_h8_n1024_d64": dict(B=4, H=8, N=1024, d=64, sigma_qk=1.0),
+    # profiling size: Q, K, V, O = 4 x 64 MiB, above the L2, a short launch
+    "b1_h64_n4096_d128": dict(B=1, H=64, N=4096, d=128, sigma_qk=1.0),
 }
+MODES = {"both": (False, True), "non-causal": (False,), "causal": (True,)}
 DEFAULT_WORKLOAD = "b1_h32_n16384_d128_qk_sigma3"
 
 
@@ -227,10 +230,10 @@ def run_reference(args, cfg):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(name, cfg, n_gpus):
+def workload_config(name, cfg, n_gpus, modes=(False, True)):
     return {"workload": name, "B": cfg["B"], "H": cfg["H"], "N": cfg["N"], "d": cfg["d"],
             "qk_sigma": cfg["sigma_qk"], "v_sigma": 1.0, "scale": "1/sqrt(d)",
-            "modes": ["non-causal", "causal"], "seed": 0,
+            "modes": ["causal" if c else "non-causal" for c in modes], "seed": 0,
             "l2": "inputs (Q,K,V = 3 x {:.0f} MiB) larger than the 126 MB L2".format(
                 cfg["B"] * cfg["H"] * cfg["N"] * cfg["d"] * 2 / 2 ** 20),
             "parallelism": f"replicas x{n_gpus} (independent (b,h) slices, no collective)"}
@@ -251,16 +254,17 @@ def run_ours(args, cfg):
     import seeded_inputs as si
 
     B, H, N, d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
+    modes = MODES[args.modes]
     bits = si.make_qkv(B, H, N, d, seed=rank, sigma_qk=cfg["sigma_qk"])
 
     def dev_tensor(b):
         return torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
 
     q, k, v = (dev_tensor(b) for b in bits)
-    o = {c: torch.empty_like(q) for c in (False, True)}
-    lse = {c: torch.empty((B, H, N), dtype=torch.float32, device=dev) for c in (False, True)}
+    o = {c: torch.empty_like(q) for c in modes}
+    lse = {c: torch.empty((B, H, N), dtype=torch.float32, device=dev) for c in modes}
     stream = torch.cuda.current_stream(dev)
-    f_step = flops(B, H, N, d, False) + flops(B, H, N, d, True)
+    f_step = sum(flops(B, H, N, d, c) for c in modes)
 
     def barrier():
         if world > 1:
@@ -277,11 +281,11 @@ def run_ours(args, cfg):
 
     # ---------------- device-resident timing, per-launch events
     for _ in range(args.warmup):
-        for c in (False, True):
+        for c in modes:
             fa.fa_fwd(q, k, v, causal=c, out=o[c], lse=lse[c])
     torch.cuda.synchronize()
     ev = {c: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)] for c in (False, True)}
+              for _ in range(args.steps)] for c in modes}
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     gpu_index = local
     with ClockSampler(gpu_index) as clk:
@@ -289,7 +293,7 @@ def run_ours(args, cfg):
         torch.cuda.synchronize()
         t_start.record(stream)
         for s in range(args.steps):
-            for c in (False, True):
+            for c in modes:
                 ev[c][s][0].record(stream)
                 fa.fa_fwd(q, k, v, causal=c, out=o[c], lse=lse[c])
                 ev[c][s][1].record(stream)
@@ -297,7 +301,7 @@ def run_ours(args, cfg):
         torch.cuda.synchronize()
         barrier()
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
-    launch_ms = {c: statistics.mean(a.elapsed_time(b) for a, b in ev[c]) for c in (False, True)}
+    launch_ms = {c: statistics.mean(a.elapsed_time(b) for a, b in ev[c]) for c in modes}
     clocks = clk.summary()
     value = world * f_step * args.steps / (elapsed_ms / 1e3) / 1e12
 
@@ -305,13 +309,13 @@ def run_ours(args, cfg):
     e2e = None
     if not args.no_e2e:
         host = [torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).pin_memory() for b in bits]
-        o_h = {c: torch.empty_like(host[0]).pin_memory() for c in (False, True)}
-        l_h = {c: torch.empty((B, H, N), dtype=torch.float32).pin_memory() for c in (False, True)}
+        o_h = {c: torch.empty_like(host[0]).pin_memory() for c in modes}
+        l_h = {c: torch.empty((B, H, N), dtype=torch.float32).pin_memory() for c in modes}
         qd, kd, vd = (torch.empty_like(q) for _ in range(3))
         e2e_steps = max(1, min(args.steps, 10))
 
         def e2e_step():
-            for c in (False, True):
+            for c in modes:
                 fa.fa_fwd_host(host[0], host[1], host[2], o_h[c], l_h[c], qd, kd, vd, o[c], lse[c],
                                causal=c)
 
@@ -335,8 +339,8 @@ def run_ours(args, cfg):
 
     # ---------------- roofline of the dominant launch (non-causal instantiation)
     peaks = load_peaks()
-    ach = {c: flops(B, H, N, d, c) / (launch_ms[c] / 1e3) / 1e12 for c in (False, True)}
-    dominant = False if launch_ms[False] >= launch_ms[True] else True
+    ach = {c: flops(B, H, N, d, c) / (launch_ms[c] / 1e3) / 1e12 for c in modes}
+    dominant = max(modes, key=lambda c: launch_ms[c])
     roofline = {"bound": "tensor", "kernel": f"fa_fwd_kernel<{d},{str(dominant).lower()}>",
                 "achieved": ach[dominant], "peak": peaks["bf16"], "unit": "TFLOP/s",
                 "frac": ach[dominant] / peaks["bf16"], "peak_source": peaks["source"] + " burst",
@@ -345,11 +349,11 @@ def run_ours(args, cfg):
                     "ms_per_launch": launch_ms[c], "tflops": ach[c],
                     "frac_of_measured_burst": ach[c] / peaks["bf16"],
                     "frac_of_measured_sustained": ach[c] / peaks["bf16_sustained"],
-                    "frac_of_datasheet_2250": ach[c] / DATASHEET_BF16_TFLOPS} for c in (False, True)}}
+                    "frac_of_datasheet_2250": ach[c] / DATASHEET_BF16_TFLOPS} for c in modes}}
 
     # ---------------- CPU baseline (rank 0, N=1 only)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.modes == "both":
         v_cpu, det = oracle_sample(bits, cfg, args.cpu_seconds)
         par = sample_parity(det["results"], o, lse, d)
         cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": det["cores"], "kind": "oracle",
@@ -362,12 +366,12 @@ def run_ours(args, cfg):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": workload_config(args.workload, cfg, world),
+            "data": "synthetic", "config": workload_config(args.workload, cfg, world, modes),
             "pct_of_peak": {"measured_burst": 100 * value / world / peaks["bf16"],
                             "measured_sustained": 100 * value / world / peaks["bf16_sustained"],
                             "datasheet_2250": 100 * value / world / DATASHEET_BF16_TFLOPS},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps * 2 * fa.launches_per_call(B, H, N, d),
+            "gpu_launches": args.steps * len(modes) * fa.launches_per_call(B, H, N, d),
             "clocks": clocks, "impl": "ours",
         }
         print(json.dumps(line), flush=True)
@@ -379,10 +383,12 @@ def run_ours(args, cfg):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--modes", choices=sorted(MODES), default="both",
+                    help="masking modes in one step (the headline uses both)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
