@@ -429,26 +429,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wait_bar(bar_kv_full + 8 * (i % C::kSlots), (i / C::kSlots) & 1, abort, p.status);
                 tc_fence_after();
             };
+            // Descriptors are built once; the start-address field (bits 0..13,
+            // address >> 4) is advanced by plain integer adds, which never carry
+            // out of the field for shared-memory addresses below 256 KiB.  This
+            // keeps the issuing thread's instruction count per MMA minimal.
+            const uint64_t desc_k = smem_desc_sw128(0, 16, 1024);
+            const uint64_t desc_v = smem_desc_sw128(0, C::kBoxBytes, 1024);
+            const uint64_t desc_q0 = desc_k + (q_smem >> 4);
+            const uint64_t desc_q1 = desc_k + ((q_smem + C::kTileBytes) >> 4);
             // S_t = Q_t K^T: K-major A and B, 128-byte swizzle, 16 columns of d per MMA.
             auto issue_s = [&](int t, uint32_t k_smem) {
+                const uint64_t a0 = t ? desc_q1 : desc_q0;
+                const uint64_t b0 = desc_k + (k_smem >> 4);
+                const uint32_t d_tmem = tmem + C::col_s(t);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-                    const uint64_t a = smem_desc_sw128(q_smem + t * C::kTileBytes + off, 16, 1024);
-                    const uint64_t b = smem_desc_sw128(k_smem + off, 16, 1024);
-                    mma_ss(tmem + C::col_s(t), a, b, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+                    mma_ss(d_tmem, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             // O_t += P_t V: P_t from TMEM (8 columns per 16 keys); V is MN-major
             // (d contiguous): 8-key groups 1024 bytes apart, 64-column halves
-            // of d one box (16 KiB) apart.
+            // of d one box (16 KiB) apart; 16 keys = 2048 bytes per MMA.
             auto issue_pv = [&](int t, uint32_t v_smem, bool acc) {
+                const uint64_t b0 = desc_v + (v_smem >> 4);
+                const uint32_t d_tmem = tmem + C::col_o(t);
+                const uint32_t a_tmem = tmem + C::col_s(t) + C::kColP;
 #pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    const uint64_t b = smem_desc_sw128(v_smem + kk * 2048, C::kBoxBytes, 1024);
-                    mma_ts(tmem + C::col_o(t), tmem + C::col_s(t) + C::kColP + kk * 8, b, idesc_o,
+                for (int kk = 0; kk < kBlockN / 16; ++kk)
+                    mma_ts(d_tmem, a_tmem + kk * 8, b0 + kk * (2048 >> 4), idesc_o,
                            (acc || kk > 0) ? 1u : 0u);
-                }
             };
 
             wait_bar(bar_q_full, 0, abort, p.status);
