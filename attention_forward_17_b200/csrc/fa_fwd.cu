@@ -138,9 +138,9 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
     p.status = dev_status;
     p.N = static_cast<int>(N);
     p.BH = static_cast<int>(BH);
-    p.n_qblk = static_cast<int>((N + 255) / 256);
+    p.n_qtile = static_cast<int>((N + fa::kBlockM - 1) / fa::kBlockM);
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-    const int64_t grid = BH * p.n_qblk;
+    const int64_t grid = BH * p.n_qtile;
     if (grid > 0x7fffffffLL) return FA_ERR_SHAPE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;

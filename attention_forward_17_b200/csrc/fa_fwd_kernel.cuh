@@ -4,32 +4,41 @@
 //   O[i, :] = sum_j softmax_j(scale * q_i . k_j  [j <= i when causal]) v_j
 //   LSE[i]  = ln sum_j exp(scale * q_i . k_j)
 // without writing the score matrix anywhere: query, key and value tiles are
-// streamed through shared memory and the softmax is updated online with a
+// streamed through on-chip memory and the softmax is updated online with a
 // running row maximum, a running normaliser and rescaling factors, while both
 // products (Q K^T and P V) run on the tensor cores ("TileLang tutorial",
 // FlashAttention section).
 //
-// Blackwell mapping (one CTA = 256 query rows of one (b, h) slice, as two
-// 128-row tiles t = 0, 1 processed in ping-pong; 384 threads, and the
-// softmax warpgroups take registers from the third warpgroup with setmaxnreg):
-//   warp 8      TMA producer: Q tiles once, then K_j / V_j tiles through a
-//               ring of shared-memory slots (mbarrier full/empty pairs).
-//   warp 9      MMA issuer (one thread): S_t = Q_t K_j^T into tensor memory
-//               (TMEM), and O_t += P_t V_j with P_t read from TMEM.
-//   warps 0-7   two softmax warpgroups; thread = query row = TMEM lane.  They
-//               read S_t from TMEM, apply the causal / length mask, keep the
-//               running max m (base-2, scaled) and sum l, rescale O_t in TMEM
-//               only when m grows by more than 2^8 (lazy rescale; the final
-//               O / l uses the same stale m, so it is exact), write P_t as
-//               bf16 into TMEM over S_t, and finally normalise and store O_t
-//               and LSE.  O is divided by the sum of the bf16-rounded weights
-//               the P V product actually used, so every O row is an exact
-//               convex combination of V rows (a one-hot row returns its V row
-//               unchanged); LSE uses the fp32 sum of the unrounded weights.
+// Blackwell mapping.  One CTA = one 128-row query tile of one (b, h) slice;
+// 384 threads in three warpgroups:
+//   warpgroups 0 and 1  softmax.  Each warp owns 16 query rows (TMEM lanes
+//               32*quarter + 16*g ..) through the 16-lane TMEM access shapes; a
+//               row's 128 scores sit in four adjacent threads, so row maxima
+//               need two shuffles and the eight softmax warps run without any
+//               barrier between them.
+//   warp 8      TMA producer: the Q tile once, then K_j and V_j tiles through
+//               one ring of shared-memory slots (mbarrier full/empty pairs).
+//   warp 9      score issuer (one thread): S_b = Q K_j^T on tcgen05, Q and K_j
+//               from shared memory, S_b into tensor memory (TMEM).
+//   warp 10     output issuer (one thread): O += P_b V_j on tcgen05, P_b from
+//               TMEM, V_j from shared memory.
+//               A thread issues one tcgen05.mma about every 48 cycles while a
+//               128x128x16 product takes 64 on the tensor pipe, so one issuing
+//               thread alone leaves the pipe idle; two keep it fed.
+//               The score tile is triple-buffered (b = j mod 3): S for steps
+//               j+1 and j+2 is computed while the softmax works on step j, and
+//               buffer b is rewritten only after the product that read its P
+//               has completed.
+// The softmax keeps the running max m (base 2, scaled) and sums l; O is
+// rescaled in TMEM only when m grows by more than 2^8 (lazy rescale: the final
+// O / l uses the same stale m, so it is exact).  O is divided by the sum of the
+// bf16-rounded weights the P V product actually used, so every O row is an
+// exact convex combination of V rows; LSE uses the fp32 sum of the unrounded
+// weights.  A share of the exponentials runs on the FMA pipe (exp2_poly2).
 //
-// TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
-// O_1 [256+D, 256+2D).  P_t (bf16, two per column) sits in the upper half of
-// S_t, columns [64,128) of that tile.
+// TMEM columns (512 allocated): S_0 [0,128), S_1 [128,256), S_2 [256,384),
+// O [384, 384+D).  P_b (bf16, two per column) sits in columns [64,128) of S_b:
+// keys 0-63 then keys 64-127.
 //
 // Every mbarrier wait is bounded in time.  A wait that gives up records
 // FA_ERR_TIMEOUT in the optional status word, marks the CTA as aborted (later
@@ -45,13 +54,16 @@
 
 namespace fa {
 
-constexpr int kThreads = 384;     // 2 softmax warpgroups + 1 warpgroup (producer, MMA, 2 spare)
-constexpr int kBlockM = 128;      // query rows per tile (= TMEM lanes)
+constexpr int kThreads = 384;     // 2 softmax warpgroups + producer, 2 MMA issuers, 1 spare
+constexpr int kSBufs = 3;         // score / probability buffers in TMEM
+constexpr int kBlockM = 128;      // query rows per CTA (= TMEM lanes)
 constexpr int kBlockN = 128;      // key rows per tile
-constexpr int kTilesPerCta = 2;   // ping-pong query tiles
 constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;       // score issuer; also allocates TMEM
+constexpr int kPvWarp = 10;       // output issuer
 constexpr int kStatusTimeout = -7;  // FA_ERR_TIMEOUT
+constexpr uint64_t kWaitLimitNs = 2000000000ull;      // 2 s
+constexpr uint64_t kWaitLimitAbortNs = 1000000ull;    // 1 ms once the CTA has aborted
 // Per-thread registers after the warpgroups rebalance (launch: 384 x 168).
 constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kRegsOther = 88;
@@ -59,52 +71,60 @@ constexpr int kRegSplitTotal = 2 * 128 * kRegsSoftmax + 128 * kRegsOther;  // 64
 // Every kEmuEvery-th pair of exponentials is evaluated on the FMA pipe by
 // polynomial instead of on the special-function unit (0 = never).
 constexpr int kEmuEvery = 4;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;      // 2 s
-constexpr uint64_t kWaitLimitAbortNs = 1000000ull;    // 1 ms once the CTA has aborted
 
 template <int D>
 struct TileCfg {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
-    static constexpr int kTileBytes = kBlockM * D * 2;      // one Q, K or V tile (bf16)
+    static constexpr int kTileBytes = kBlockN * D * 2;      // one K or V tile (bf16)
     static constexpr int kBoxes = D / 64;                   // 64-column (128-byte) TMA boxes
     static constexpr int kBoxBytes = 128 * 128;             // 128 rows x 128 bytes
-    static constexpr int kSlots = (D == 128) ? 4 : 8;       // K/V ring depth
+    static constexpr int kSlots = (D == 128) ? 5 : 8;       // K/V ring depth
     static constexpr int kQOff = 0;
-    static constexpr int kSlotOff = kTilesPerCta * kTileBytes;
+    static constexpr int kSlotOff = kTileBytes;             // after the Q tile
     static constexpr int kBarOff = kSlotOff + kSlots * kTileBytes;
-    static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBarOff + 512;
-    __host__ __device__ static constexpr uint32_t col_s(int t) { return 128u * t; }
-    __host__ __device__ static constexpr uint32_t col_o(int t) { return 256u + D * t; }
-    static constexpr uint32_t kColP = 64;                   // offset of P inside S
+    static constexpr int kRedOff = kBarOff + 512;           // row-max / sum exchange
+    static constexpr int kSmemBytes = 1024 /* alignment slack */ + kRedOff + 4 * 2 * 128 * 4;
+    __host__ __device__ static constexpr uint32_t col_s(int b) { return 128u * b; }
+    static constexpr uint32_t kColO = 128 * kSBufs;
+    static constexpr uint32_t kColP = 64;                   // offset of P inside S_b
     static constexpr uint32_t kTmemCols = 512;
 };
 
 template <int kSlots>
 struct alignas(8) Barriers {
-    uint64_t q_full[2];
     uint64_t kv_full[kSlots];
     uint64_t kv_empty[kSlots];
-    uint64_t s_full[2];
-    uint64_t p_full[2];
-    uint64_t o_full[2];
-    uint64_t mma_done;
+    uint64_t q_full;            // Q tile landed in shared memory
+    uint64_t s_full[kSBufs];    // S_b computed
+    uint64_t p_full[kSBufs];    // P_b written (and O rescaled)
+    uint64_t pv_done[kSBufs];   // O += P_b V of the latest use of buffer b completed
+    uint64_t o_full;            // every product done
     uint32_t tmem_base;
     volatile uint32_t abort;
 };
 
 struct FwdParams {
-    __nv_bfloat16* o;     // [BH, N, D]
-    float* lse;           // [BH, N]
-    int* status;          // optional device status word (may be null)
+    __nv_bfloat16* o;        // [BH, N, D]
+    float* lse;              // [BH, N]
+    int* status;             // optional device status word (may be null)
     int N;
     int BH;
-    int n_qblk;           // ceil(N / 256)
-    float scale_log2;     // scale * log2(e)
+    int n_qtile;             // ceil(N / 128)
+    float scale_log2;        // scale * log2(e)
 };
+
+// Load sequence of the K/V ring: K_0 .. K_{min(3,n)-1}, then for each step t
+// V_t followed by K_{t+3} (while t + 3 < n).  Each load's slot is released by
+// the issuer that consumes it; a release only ever depends on loads earlier in
+// the sequence, so the ring cannot deadlock.
+__device__ __forceinline__ int load_index_k(int m) { return m < kSBufs ? m : 2 * m - kSBufs + 1; }
+__device__ __forceinline__ int load_index_v(int t, int n) {
+    return min(kSBufs, n) + t + min(t, max(0, n - kSBufs));
+}
 
 // ---------------------------------------------------------------- bounded waits
 __device__ __forceinline__ void wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
-                                       int* status) {
+                                          int* status) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return;
@@ -169,41 +189,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_addr);
     auto* bars = reinterpret_cast<Barriers<C::kSlots>*>(smem + C::kBarOff);
+    // final per-row statistics handed to the epilogue: m [0,128), l [128,256), l-hat [256,384)
+    float* red = reinterpret_cast<float*>(smem + C::kRedOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     // Work item: CTAs of one (b, h) slice are adjacent in launch order so the
-    // slice's K/V stay in L2; under the causal mask the longest q-blocks of a
-    // slice launch first.
-    const int bh = blockIdx.x / p.n_qblk;
-    const int qi = blockIdx.x % p.n_qblk;
-    const int qb = CAUSAL ? (p.n_qblk - 1 - qi) : qi;
-    const int q0 = qb * (kBlockM * kTilesPerCta);
+    // slice's K/V stay in L2; under the causal mask the longest query tiles of
+    // a slice launch first.
+    const int bh = blockIdx.x / p.n_qtile;
+    const int qi = blockIdx.x % p.n_qtile;
+    const int qt = CAUSAL ? (p.n_qtile - 1 - qi) : qi;
+    const int q0 = qt * kBlockM;
     const int n_kv_all = (p.N + kBlockN - 1) / kBlockN;
-    const int n_kv = CAUSAL ? min(n_kv_all, 2 * qb + 2) : n_kv_all;
+    const int n_kv = CAUSAL ? min(n_kv_all, qt + 1) : n_kv_all;
 
-    const uint32_t bar_q_full = smem_u32(&bars->q_full[0]);
     const uint32_t bar_kv_full = smem_u32(&bars->kv_full[0]);
     const uint32_t bar_kv_empty = smem_u32(&bars->kv_empty[0]);
+    const uint32_t bar_q_full = smem_u32(&bars->q_full);
     const uint32_t bar_s_full = smem_u32(&bars->s_full[0]);
     const uint32_t bar_p_full = smem_u32(&bars->p_full[0]);
-    const uint32_t bar_o_full = smem_u32(&bars->o_full[0]);
-    const uint32_t bar_mma_done = smem_u32(&bars->mma_done);
+    const uint32_t bar_pv_done = smem_u32(&bars->pv_done[0]);
+    const uint32_t bar_o_full = smem_u32(&bars->o_full);
     volatile uint32_t* abort = &bars->abort;
 
     if (threadIdx.x == 0) {
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(bar_q_full + 8 * t, 1);
-            mbar_init(bar_s_full + 8 * t, 1);
-            mbar_init(bar_p_full + 8 * t, kBlockM);
-            mbar_init(bar_o_full + 8 * t, 1);
-        }
         for (int s = 0; s < C::kSlots; ++s) {
             mbar_init(bar_kv_full + 8 * s, 1);
             mbar_init(bar_kv_empty + 8 * s, 1);
         }
-        mbar_init(bar_mma_done, 1);
+        mbar_init(bar_q_full, 1);
+        for (int b = 0; b < kSBufs; ++b) {
+            mbar_init(bar_s_full + 8 * b, 1);
+            mbar_init(bar_p_full + 8 * b, 256);
+            mbar_init(bar_pv_done + 8 * b, 1);
+        }
+        mbar_init(bar_o_full, 1);
         bars->abort = 0u;
         fence_barrier_init();
     }
@@ -224,135 +246,198 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < 8) {
         regs_increase<kRegsSoftmax>();
         // ============================================================ softmax
-        const int t = warp >> 2;                  // query tile of this warpgroup
-        const int r = threadIdx.x & 127;          // row within the tile = TMEM lane
-        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t t_s = tmem + lane_off + C::col_s(t);
-        const uint32_t t_p = t_s + C::kColP;
-        const uint32_t t_o = tmem + lane_off + C::col_o(t);
-        const int tile_row0 = q0 + t * kBlockM;
-        const int row = tile_row0 + r;
+        // Warp (g, quarter) owns the 16 tile rows L .. L+15, L = 32*quarter +
+        // 16*g, through the 16-lane TMEM access shapes: thread t holds rows
+        // ra = L + t/4 and rb = ra + 8, keys 8m + 2(t%4) + {0,1} (m = 0..15) of
+        // each score tile, so a row's 128 keys live in four adjacent threads.
+        const int quarter = warp & 3;
+        const int g = warp >> 2;
+        const int L = 32 * quarter + 16 * g;
+        const int ra = L + (lane >> 2), rb = ra + 8;
+        const int kq = 2 * (lane & 3);            // key offset inside each 8-key chunk
+        const uint32_t lane_w = static_cast<uint32_t>(L) << 16;
         const float c = p.scale_log2;
-
-        float m_run = -INFINITY;   // running max of scale*log2(e)*s (possibly stale by < 8)
-        float l_run = 0.f;         // running sum of 2^(c*s - m_run), fp32 (for LSE)
-        float lh_run = 0.f;        // running sum of the same weights rounded to bf16 (for O)
-
         const uint64_t c2 = f2(c, c);
-        for (int j = 0; j < n_kv; ++j) {
-            wait_bar(bar_s_full + 8 * t, j & 1, abort, p.status);
-            tc_fence_after();
-            uint32_t s[4][32];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) tmem_ld32(t_s + 32 * q, s[q]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int q = 0; q < 4; ++q) reg_fence32(s[q]);
 
-            const int k0 = j * kBlockN;
-            const bool masked = (k0 + kBlockN > p.N) || (CAUSAL && k0 + kBlockN - 1 > tile_row0);
+        float m_a = -INFINITY, m_b = -INFINITY;   // running max of c*s per row (stale by < 8)
+        float l_a = 0.f, l_b = 0.f;               // fp32 sums of 2^(c*s - m) (for LSE), this thread's keys
+        float lh_a = 0.f, lh_b = 0.f;             // the same weights rounded to bf16 (for O)
+
+        for (int j = 0; j < n_kv; ++j) {
+            const int bb = j % kSBufs;
+            const uint32_t t_s = tmem + lane_w + C::col_s(bb);
+            wait_bar(bar_s_full + 8 * bb, (j / kSBufs) & 1, abort, p.status);
+            tc_fence_after();
+            uint32_t s[64];
+            tmem_ld16x256b_x16(t_s, s);
+            tmem_wait_ld();
+            reg_fence64(s);
+
+            const bool masked =
+                (j * kBlockN + kBlockN > p.N) || (CAUSAL && j * kBlockN + kBlockN - 1 > q0);
             if (masked) {
-                const int lim = (CAUSAL ? min(p.N, row + 1) : p.N) - k0;
+                const int lim_a = (CAUSAL ? min(p.N, q0 + ra + 1) : p.N) - j * kBlockN;
+                const int lim_b = (CAUSAL ? min(p.N, q0 + rb + 1) : p.N) - j * kBlockN;
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
+                for (int m = 0; m < 16; ++m)
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (32 * q + i >= lim) s[q][i] = __float_as_uint(-INFINITY);
+                    for (int e = 0; e < 2; ++e) {
+                        const int key = 8 * m + kq + e;
+                        if (key >= lim_a) s[4 * m + e] = __float_as_uint(-INFINITY);
+                        if (key >= lim_b) s[4 * m + 2 + e] = __float_as_uint(-INFINITY);
+                    }
             }
-            // row max: eight independent 3-input max chains
-            float mx[8];
+            // row maxima: 32 values per row in this thread, then across the 4 threads
+            float xa0 = fmaxf(__uint_as_float(s[0]), __uint_as_float(s[1]));
+            float xb0 = fmaxf(__uint_as_float(s[2]), __uint_as_float(s[3]));
+            float xa1 = fmaxf(__uint_as_float(s[4]), __uint_as_float(s[5]));
+            float xb1 = fmaxf(__uint_as_float(s[6]), __uint_as_float(s[7]));
 #pragma unroll
-            for (int a = 0; a < 8; ++a) mx[a] = __uint_as_float(s[a >> 1][(a & 1) * 16]);
-#pragma unroll
-            for (int a = 0; a < 8; ++a) {
-                const int q = a >> 1, b0 = (a & 1) * 16;
-#pragma unroll
-                for (int i = 1; i < 15; i += 2)
-                    mx[a] = max3f(mx[a], __uint_as_float(s[q][b0 + i]), __uint_as_float(s[q][b0 + i + 1]));
-                mx[a] = fmaxf(mx[a], __uint_as_float(s[q][b0 + 15]));
+            for (int m = 2; m < 16; m += 2) {
+                xa0 = max3f(xa0, __uint_as_float(s[4 * m]), __uint_as_float(s[4 * m + 1]));
+                xb0 = max3f(xb0, __uint_as_float(s[4 * m + 2]), __uint_as_float(s[4 * m + 3]));
+                xa1 = max3f(xa1, __uint_as_float(s[4 * m + 4]), __uint_as_float(s[4 * m + 5]));
+                xb1 = max3f(xb1, __uint_as_float(s[4 * m + 6]), __uint_as_float(s[4 * m + 7]));
             }
-            const float m_new =
-                max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c;
-            const bool grow = m_new > m_run + 8.0f;
-            float alpha = 1.f;
-            if (grow) {
-                alpha = ex2_approx(m_run - m_new);
-                m_run = m_new;
-                l_run *= alpha;
-                lh_run *= alpha;
+            float mxa = fmaxf(xa0, xa1), mxb = fmaxf(xb0, xb1);
+            mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
+            mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
+            mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
+            mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
+            const float mna = mxa * c, mnb = mxb * c;
+            const bool ga = mna > m_a + 8.0f, gb = mnb > m_b + 8.0f;
+            float alpha_a = 1.f, alpha_b = 1.f;
+            if (ga) {
+                alpha_a = ex2_approx(m_a - mna);
+                m_a = mna;
+                l_a *= alpha_a;
+                lh_a *= alpha_a;
             }
-            if (j > 0 && __any_sync(0xffffffffu, grow)) {
-                // O_t holds sum_{j' < j} P V with the old reference max: scale
-                // it by 2^(m_old - m_new).  The commit that signalled S_t(j)
-                // also covers the P V product of step j-1.
-#pragma unroll 1
-                for (int q = 0; q < D / 32; ++q) {
+            if (gb) {
+                alpha_b = ex2_approx(m_b - mnb);
+                m_b = mnb;
+                l_b *= alpha_b;
+                lh_b *= alpha_b;
+            }
+            if (j > 0 && __any_sync(0xffffffffu, ga || gb)) {
+                // O holds sum_{j' < j} P V with the old reference maxima: scale
+                // these 16 rows by 2^(m_old - m_new) once the product of step
+                // j-1 has landed.
+                wait_bar(bar_pv_done + 8 * ((j - 1) % kSBufs), ((j - 1) / kSBufs) & 1, abort,
+                         p.status);
+                tc_fence_after();
+                const uint32_t t_o = tmem + lane_w + C::kColO;
+                if constexpr (D == 128) {
+                    uint32_t o[64];
+                    tmem_ld16x256b_x16(t_o, o);
+                    tmem_wait_ld();
+                    reg_fence64(o);
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        o[4 * m] = __float_as_uint(__uint_as_float(o[4 * m]) * alpha_a);
+                        o[4 * m + 1] = __float_as_uint(__uint_as_float(o[4 * m + 1]) * alpha_a);
+                        o[4 * m + 2] = __float_as_uint(__uint_as_float(o[4 * m + 2]) * alpha_b);
+                        o[4 * m + 3] = __float_as_uint(__uint_as_float(o[4 * m + 3]) * alpha_b);
+                    }
+                    tmem_st16x256b_x16(t_o, o);
+                } else {
                     uint32_t o[32];
-                    tmem_ld32(t_o + 32 * q, o);
+                    tmem_ld16x256b_x8(t_o, o);
                     tmem_wait_ld();
                     reg_fence32(o);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(t_o + 32 * q, o);
+                    for (int m = 0; m < 8; ++m) {
+                        o[4 * m] = __float_as_uint(__uint_as_float(o[4 * m]) * alpha_a);
+                        o[4 * m + 1] = __float_as_uint(__uint_as_float(o[4 * m + 1]) * alpha_a);
+                        o[4 * m + 2] = __float_as_uint(__uint_as_float(o[4 * m + 2]) * alpha_b);
+                        o[4 * m + 3] = __float_as_uint(__uint_as_float(o[4 * m + 3]) * alpha_b);
+                    }
+                    tmem_st16x256b_x8(t_o, o);
                 }
             }
-            const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-            const uint64_t negm2 = f2(-m_use, -m_use);
-            // p = 2^(c*s - m): pairs of columns through packed FMAs; sums of the
-            // fp32 weights (l, for LSE) and of their bf16 roundings (for O)
-            uint64_t l2a = 0, l2b = 0, h2a = 0, h2b = 0;
+            const float ua = (m_a == -INFINITY) ? 0.f : m_a;
+            const float ub = (m_b == -INFINITY) ? 0.f : m_b;
+            const uint64_t nega = f2(-ua, -ua), negb = f2(-ub, -ub);
+            // p = 2^(c*s - m) pairwise through packed FMAs; sums of the fp32
+            // weights (for LSE) and of their bf16 roundings (for O).  P word
+            // 2m / 2m+1 = keys 8m + kq + {0,1} of row a / row b, which is the
+            // 16x128b store layout at column 4m + t%4 of the P region.
+            uint64_t la2 = 0, lb2 = 0, ha2 = 0, hb2 = 0;
+            uint32_t pk[32];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int col = 64 * h + 2 * i;
-                    const uint64_t x2 = fma2(f2(__uint_as_float(s[col >> 5][col & 31]),
-                                                __uint_as_float(s[col >> 5][(col & 31) + 1])),
-                                             c2, negm2);
-                    float x0, x1;
-                    f2_split(x2, x0, x1);
-                    float p0, p1;
-                    if (kEmuEvery > 0 && (i % kEmuEvery) == kEmuEvery - 1) {
-                        exp2_poly2(x0, x1, p0, p1);
-                    } else {
-                        p0 = ex2_approx(x0);
-                        p1 = ex2_approx(x1);
-                    }
-                    const uint32_t w = pack_bf16x2(p0, p1);
-                    const uint64_t pr = f2(p0, p1);
-                    const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-                    if (i & 1) {
-                        l2b = add2(l2b, pr);
-                        h2b = add2(h2b, ph);
-                    } else {
-                        l2a = add2(l2a, pr);
-                        h2a = add2(h2a, ph);
-                    }
-                    pk[i] = w;
+            for (int i = 0; i < 32; ++i) {
+                const int m = i >> 1;
+                const bool row_b = i & 1;
+                const uint64_t x2 = fma2(f2(__uint_as_float(s[4 * m + 2 * row_b]),
+                                            __uint_as_float(s[4 * m + 2 * row_b + 1])),
+                                         c2, row_b ? negb : nega);
+                float x0, x1;
+                f2_split(x2, x0, x1);
+                float p0, p1;
+                if (kEmuEvery > 0 && (i % kEmuEvery) == kEmuEvery - 1) {
+                    exp2_poly2(x0, x1, p0, p1);
+                } else {
+                    p0 = ex2_approx(x0);
+                    p1 = ex2_approx(x1);
                 }
-                tmem_st32(t_p + 32 * h, pk);
+                const uint32_t w = pack_bf16x2(p0, p1);
+                const uint64_t pr = f2(p0, p1);
+                const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+                if (row_b) {
+                    lb2 = add2(lb2, pr);
+                    hb2 = add2(hb2, ph);
+                } else {
+                    la2 = add2(la2, pr);
+                    ha2 = add2(ha2, ph);
+                }
+                pk[i] = w;
             }
-            float la0, la1, lb0, lb1, ha0, ha1, hb0, hb1;
-            f2_split(l2a, la0, la1);
-            f2_split(l2b, lb0, lb1);
-            f2_split(h2a, ha0, ha1);
-            f2_split(h2b, hb0, hb1);
-            l_run += (la0 + la1) + (lb0 + lb1);
-            lh_run += (ha0 + ha1) + (hb0 + hb1);
+            tmem_st16x128b_x16(t_s + C::kColP, pk);
+            float u0, u1;
+            f2_split(la2, u0, u1);
+            l_a += u0 + u1;
+            f2_split(lb2, u0, u1);
+            l_b += u0 + u1;
+            f2_split(ha2, u0, u1);
+            lh_a += u0 + u1;
+            f2_split(hb2, u0, u1);
+            lh_b += u0 + u1;
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar_p_full + 8 * t);
+            mbar_arrive(bar_p_full + 8 * bb);
         }
 
         // ------------------------------------------------------------ epilogue
-        wait_bar(bar_o_full + 8 * t, 0, abort, p.status);
+        // Row totals over the four threads of each row, published per tile row
+        // for the 32-lane epilogue layout (thread = row).
+#pragma unroll
+        for (int sh = 1; sh <= 2; sh <<= 1) {
+            l_a += __shfl_xor_sync(0xffffffffu, l_a, sh);
+            l_b += __shfl_xor_sync(0xffffffffu, l_b, sh);
+            lh_a += __shfl_xor_sync(0xffffffffu, lh_a, sh);
+            lh_b += __shfl_xor_sync(0xffffffffu, lh_b, sh);
+        }
+        if ((lane & 3) == 0) {
+            red[ra] = m_a;
+            red[128 + ra] = l_a;
+            red[256 + ra] = lh_a;
+            red[rb] = m_b;
+            red[128 + rb] = l_b;
+            red[256 + rb] = lh_b;
+        }
+        named_barrier_sync(1 + quarter, 64);
+        const int r = 32 * quarter + lane;        // epilogue row of this thread
+        const int row = q0 + r;
+        const float m_r = red[r], l_r = red[128 + r], lh_r = red[256 + r];
+        wait_bar(bar_o_full, 0, abort, p.status);
         tc_fence_after();
         const bool valid = row < p.N;
-        const float inv_l = lh_run > 0.f ? 1.f / lh_run : 0.f;
-        __nv_bfloat16* orow = p.o + (static_cast<int64_t>(bh) * p.N + row) * D;
+        const float inv_l = lh_r > 0.f ? 1.f / lh_r : 0.f;
+        __nv_bfloat16* orow = p.o + (static_cast<int64_t>(bh) * p.N + row) * D + g * (D / 2);
+        const uint32_t t_o =
+            tmem + (static_cast<uint32_t>(32 * quarter) << 16) + C::kColO + g * (D / 2);
 #pragma unroll 1
-        for (int q = 0; q < D / 32; ++q) {
+        for (int q = 0; q < D / 64; ++q) {
             uint32_t o[32];
             tmem_ld32(t_o + 32 * q, o);
             tmem_wait_ld();
@@ -362,16 +447,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                     uint4 w;
-                    w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
-                    w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
-                    w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
-                    w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+                    w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l,
+                                      __uint_as_float(o[8 * v + 1]) * inv_l);
+                    w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l,
+                                      __uint_as_float(o[8 * v + 3]) * inv_l);
+                    w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l,
+                                      __uint_as_float(o[8 * v + 5]) * inv_l);
+                    w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l,
+                                      __uint_as_float(o[8 * v + 7]) * inv_l);
                     dst[v] = w;
                 }
             }
         }
-        if (valid) {
-            float lse = l_run > 0.f ? (m_run + lg2_approx(l_run)) * 0.69314718055994531f : -INFINITY;
+        if (valid && g == 0) {
+            float lse = l_r > 0.f ? (m_r + lg2_approx(l_r)) * 0.69314718055994531f : -INFINITY;
             if (*abort) lse = __int_as_float(0x7fc00000);
             p.lse[static_cast<int64_t>(bh) * p.N + row] = lse;
         }
@@ -381,48 +470,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint64_t pol_q = policy_evict_first();
             const uint64_t pol_kv = policy_evict_last();
-            const uint32_t q_smem = base + C::kQOff;
             const uint32_t slot_smem = base + C::kSlotOff;
-            auto load_q = [&](int t) {
-                mbar_arrive_expect_tx(bar_q_full + 8 * t, C::kTileBytes);
+            mbar_arrive_expect_tx(bar_q_full, C::kTileBytes);
 #pragma unroll
-                for (int b = 0; b < C::kBoxes; ++b)
-                    tma_load_3d(q_smem + t * C::kTileBytes + b * C::kBoxBytes, &tm_q, 64 * b,
-                                q0 + t * kBlockM, bh, bar_q_full + 8 * t, pol_q);
-            };
-            // load index i: K_{i/2} for even i, V_{i/2} for odd i
-            auto load_kv = [&](int i) {
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+                tma_load_3d(base + C::kQOff + bx * C::kBoxBytes, &tm_q, 64 * bx, q0, bh, bar_q_full, pol_q);
+            int i = 0;
+            auto load = [&](bool is_v, int tile) {
                 const int slot = i % C::kSlots;
                 const int use = i / C::kSlots;
                 if (use > 0) wait_bar(bar_kv_empty + 8 * slot, (use - 1) & 1, abort, p.status);
-                const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
+                const CUtensorMap* map = is_v ? &tm_v : &tm_k;
                 mbar_arrive_expect_tx(bar_kv_full + 8 * slot, C::kTileBytes);
 #pragma unroll
-                for (int b = 0; b < C::kBoxes; ++b)
-                    tma_load_3d(slot_smem + slot * C::kTileBytes + b * C::kBoxBytes, map, 64 * b,
-                                (i >> 1) * kBlockN, bh, bar_kv_full + 8 * slot, pol_kv);
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                    tma_load_3d(slot_smem + slot * C::kTileBytes + bx * C::kBoxBytes, map, 64 * bx,
+                                tile * kBlockN, bh, bar_kv_full + 8 * slot, pol_kv);
+                ++i;
             };
-            load_q(0);
-            load_kv(0);
-            load_q(1);
-            for (int i = 1; i < 2 * n_kv; ++i) load_kv(i);
-            // Every load above is waited for by the MMA issuer; in an aborted
+            for (int m = 0; m < kSBufs && m < n_kv; ++m) load(false, m);
+            for (int t = 0; t < n_kv; ++t) {
+                load(true, t);
+                if (t + kSBufs < n_kv) load(false, t + kSBufs);
+            }
+            // Every load above is waited for by an MMA issuer; in an aborted
             // CTA make sure none is still landing in shared memory at exit.
             if (*abort) {
-                for (int i = max(0, 2 * n_kv - C::kSlots); i < 2 * n_kv; ++i)
-                    wait_bar(bar_kv_full + 8 * (i % C::kSlots), (i / C::kSlots) & 1, abort, p.status);
+                for (int k = max(0, 2 * n_kv - C::kSlots); k < 2 * n_kv; ++k)
+                    wait_bar(bar_kv_full + 8 * (k % C::kSlots), (k / C::kSlots) & 1, abort, p.status);
                 wait_bar(bar_q_full, 0, abort, p.status);
-                wait_bar(bar_q_full + 8, 0, abort, p.status);
             }
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kMmaWarp || warp == kPvWarp) {
         regs_decrease<kRegsOther>();
-        // ============================================================ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false);
-            constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, true);
-            const uint32_t q_smem = base + C::kQOff;
             const uint32_t slot_smem = base + C::kSlotOff;
             auto slot_addr = [&](int i) { return slot_smem + (i % C::kSlots) * C::kTileBytes; };
             auto wait_kv = [&](int i) {
@@ -431,73 +513,61 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             // Descriptors are built once; the start-address field (bits 0..13,
             // address >> 4) is advanced by plain integer adds, which never carry
-            // out of the field for shared-memory addresses below 256 KiB.  This
-            // keeps the issuing thread's instruction count per MMA minimal.
-            const uint64_t desc_k = smem_desc_sw128(0, 16, 1024);
-            const uint64_t desc_v = smem_desc_sw128(0, C::kBoxBytes, 1024);
-            const uint64_t desc_q0 = desc_k + (q_smem >> 4);
-            const uint64_t desc_q1 = desc_k + ((q_smem + C::kTileBytes) >> 4);
-            // S_t = Q_t K^T: K-major A and B, 128-byte swizzle, 16 columns of d per MMA.
-            auto issue_s = [&](int t, uint32_t k_smem) {
-                const uint64_t a0 = t ? desc_q1 : desc_q0;
-                const uint64_t b0 = desc_k + (k_smem >> 4);
-                const uint32_t d_tmem = tmem + C::col_s(t);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
-                    mma_ss(d_tmem, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
-                }
-            };
-            // O_t += P_t V: P_t from TMEM (8 columns per 16 keys); V is MN-major
-            // (d contiguous): 8-key groups 1024 bytes apart, 64-column halves
-            // of d one box (16 KiB) apart; 16 keys = 2048 bytes per MMA.
-            auto issue_pv = [&](int t, uint32_t v_smem, bool acc) {
-                const uint64_t b0 = desc_v + (v_smem >> 4);
-                const uint32_t d_tmem = tmem + C::col_o(t);
-                const uint32_t a_tmem = tmem + C::col_s(t) + C::kColP;
-#pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk)
-                    mma_ts(d_tmem, a_tmem + kk * 8, b0 + kk * (2048 >> 4), idesc_o,
-                           (acc || kk > 0) ? 1u : 0u);
-            };
-
-            wait_bar(bar_q_full, 0, abort, p.status);
-            wait_kv(0);
-            issue_s(0, slot_addr(0));
-            mma_commit(bar_s_full);
-            wait_bar(bar_q_full + 8, 0, abort, p.status);
-            tc_fence_after();
-            issue_s(1, slot_addr(0));
-            mma_commit(bar_s_full + 8);
-            mma_commit(bar_kv_empty + 8 * (0 % C::kSlots));
-            for (int j = 0; j < n_kv; ++j) {
-                const int iv = 2 * j + 1, ik = 2 * j + 2;
-                const bool more = j + 1 < n_kv;
-                wait_kv(iv);
-                wait_bar(bar_p_full, j & 1, abort, p.status);
+            // out of the field for shared-memory addresses below 256 KiB.
+            if (warp == kMmaWarp) {
+                // ==================================================== score issuer
+                // S_b = Q K^T: Q and K K-major in shared memory, 128-byte
+                // swizzle, 16 columns of d per MMA.
+                constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false);
+                const uint64_t desc_k = smem_desc_sw128(0, 16, 1024);
+                const uint64_t a0 = desc_k + ((base + C::kQOff) >> 4);
+                wait_bar(bar_q_full, 0, abort, p.status);
                 tc_fence_after();
-                issue_pv(0, slot_addr(iv), j > 0);
-                if (more) {
+                for (int m = 0; m < n_kv; ++m) {
+                    const int b = m % kSBufs;
+                    if (m >= kSBufs) {
+                        // buffer b still holds P of step m - 3 until its product is done
+                        wait_bar(bar_pv_done + 8 * b, ((m - kSBufs) / kSBufs) & 1, abort, p.status);
+                        tc_fence_after();
+                    }
+                    const int ik = load_index_k(m);
                     wait_kv(ik);
-                    issue_s(0, slot_addr(ik));
-                    mma_commit(bar_s_full);
-                } else {
-                    mma_commit(bar_o_full);
-                }
-                wait_bar(bar_p_full + 8, j & 1, abort, p.status);
-                tc_fence_after();
-                issue_pv(1, slot_addr(iv), j > 0);
-                mma_commit(bar_kv_empty + 8 * (iv % C::kSlots));
-                if (more) {
-                    issue_s(1, slot_addr(ik));
-                    mma_commit(bar_s_full + 8);
+                    const uint64_t b0 = desc_k + (slot_addr(ik) >> 4);
+                    const uint32_t d_tmem = tmem + C::col_s(b);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+                        mma_ss(d_tmem, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar_s_full + 8 * b);
                     mma_commit(bar_kv_empty + 8 * (ik % C::kSlots));
-                } else {
-                    mma_commit(bar_o_full + 8);
                 }
+            } else {
+                // ==================================================== output issuer
+                // O += P_b V: P_b from TMEM (8 columns per 16 keys); V is
+                // MN-major (d contiguous): 8-key groups 1024 bytes apart,
+                // 64-column halves of d one box (16 KiB) apart; 16 keys = 2048
+                // bytes per MMA.
+                constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, true);
+                const uint64_t desc_v = smem_desc_sw128(0, C::kBoxBytes, 1024);
+                for (int t = 0; t < n_kv; ++t) {
+                    const int b = t % kSBufs;
+                    const int iv = load_index_v(t, n_kv);
+                    wait_kv(iv);
+                    wait_bar(bar_p_full + 8 * b, (t / kSBufs) & 1, abort, p.status);
+                    tc_fence_after();
+                    const uint64_t b0 = desc_v + (slot_addr(iv) >> 4);
+                    const uint32_t a_tmem = tmem + C::col_s(b) + C::kColP;
+#pragma unroll
+                    for (int kk = 0; kk < kBlockN / 16; ++kk)
+                        mma_ts(tmem + C::kColO, a_tmem + kk * 8, b0 + kk * (2048 >> 4), idesc_o,
+                               (t > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(bar_pv_done + 8 * b);
+                    mma_commit(bar_kv_empty + 8 * (iv % C::kSlots));
+                }
+                mma_commit(bar_o_full);
+                wait_bar(bar_o_full, 0, abort, p.status);
             }
-            mma_commit(bar_mma_done);
-            wait_bar(bar_mma_done, 0, abort, p.status);
         }
         __syncwarp();
     } else {
