@@ -52,6 +52,8 @@ def _load():
     lib.fa_fwd_host.argtypes = [_vp] * 10 + [_i64, _i64, _i64, _i64, ctypes.c_int, ctypes.c_float,
                                             _vp]
     lib.fa_fwd_host.restype = ctypes.c_int
+    lib.fa_selftest_wait_timeout.argtypes = [_vp, _i64, ctypes.c_int, _vp]
+    lib.fa_selftest_wait_timeout.restype = ctypes.c_int
     lib.fa_fwd_launches.argtypes = [_i64, _i64, _i64, _i64]
     lib.fa_fwd_launches.restype = ctypes.c_int
     lib.fa_strerror.argtypes = [ctypes.c_int]
@@ -163,3 +165,13 @@ def fa_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal: bo
                              float(scale), s)
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd_host")
+
+
+def selftest_wait_timeout(status, limit_us: int, arrive: bool = False, stream=None):
+    """Run the bounded-wait self-test kernel; `status` is an int32 CUDA tensor (one element)."""
+    import torch
+    s = (stream if stream is not None else torch.cuda.current_stream(status.device)).cuda_stream
+    with torch.cuda.device(status.device):
+        rc = lib.fa_selftest_wait_timeout(status.data_ptr(), int(limit_us), int(bool(arrive)), s)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_selftest_wait_timeout")

@@ -189,6 +189,16 @@ int fa_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, fl
     return FA_OK;
 }
 
+int fa_selftest_wait_timeout(int* dev_status, int64_t limit_us, int arrive, void* stream) {
+    if (!dev_status) return FA_ERR_NULL;
+    if (limit_us < 1 || limit_us > 10000000) return FA_ERR_SHAPE;
+    int rc = current_device_ready();
+    if (rc != FA_OK) return rc;
+    fa::fa_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        dev_status, static_cast<uint64_t>(limit_us) * 1000ull, arrive ? 1 : 0);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 int fa_fwd_launches(int64_t B, int64_t H, int64_t N, int64_t d) {
     (void)d;
     return (B > 0 && H > 0 && N > 0) ? 1 : 0;

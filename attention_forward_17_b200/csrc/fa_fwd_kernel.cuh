@@ -70,7 +70,20 @@ constexpr uint32_t kRegsOther = 88;
 constexpr int kRegSplitTotal = 2 * 128 * kRegsSoftmax + 128 * kRegsOther;  // 64512 = 384 x 168
 // Every kEmuEvery-th pair of exponentials is evaluated on the FMA pipe by
 // polynomial instead of on the special-function unit (0 = never).
-constexpr int kEmuEvery = 4;
+#ifndef FA_EMU_EVERY
+#define FA_EMU_EVERY 4
+#endif
+constexpr int kEmuEvery = FA_EMU_EVERY;
+// Sum the bf16-rounded weights with mixed-precision adds that read the 16-bit
+// halves directly (1) or by widening the halves to fp32 first (0).
+#ifndef FA_LHAT_MIXED_ADD
+#define FA_LHAT_MIXED_ADD 0
+#endif
+// Evaluate the exponentials of a tile in separate passes (all exponents, then
+// all exponentials in place, then packing and sums) instead of pair by pair.
+#ifndef FA_SOFTMAX_PHASED
+#define FA_SOFTMAX_PHASED 1
+#endif
 
 template <int D>
 struct TileCfg {
@@ -123,13 +136,16 @@ __device__ __forceinline__ int load_index_v(int t, int n) {
 }
 
 // ---------------------------------------------------------------- bounded waits
+// Polls the mbarrier phase until it completes or `limit_ns` (globaltimer)
+// passes; on time-out marks the CTA aborted and records FA_ERR_TIMEOUT.  Once
+// aborted, further waits give up after `limit_abort_ns`.
 __device__ __forceinline__ void wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
-                                          int* status) {
+                                          int* status, uint64_t limit_ns, uint64_t limit_abort_ns) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return;
         if ((it & 31u) == 0) {
-            const uint64_t limit = *abort ? kWaitLimitAbortNs : kWaitLimitNs;
+            const uint64_t limit = *abort ? limit_abort_ns : limit_ns;
             if (global_timer_ns() - t0 > limit) {
                 if (!*abort) {
                     *abort = 1u;
@@ -143,7 +159,27 @@ __device__ __forceinline__ void wait_slow(uint32_t bar, uint32_t parity, volatil
 
 __device__ __forceinline__ void wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
                                          int* status) {
-    if (!mbar_try_wait(bar, parity)) wait_slow(bar, parity, abort, status);
+    if (!mbar_try_wait(bar, parity))
+        wait_slow(bar, parity, abort, status, kWaitLimitNs, kWaitLimitAbortNs);
+}
+
+// Exercises the bounded wait on an mbarrier that nothing ever arrives at: the
+// wait must give up after `limit_ns` and leave FA_ERR_TIMEOUT in *status.
+// With `arrive` set, one thread completes the phase first and the wait must
+// return at once with *status untouched.  One CTA of 32 threads.
+__global__ void fa_wait_selftest_kernel(int* status, uint64_t limit_ns, int arrive) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0u;
+        fence_barrier_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0 && arrive) mbar_arrive(smem_u32(&bar));
+    __syncwarp();
+    if (!mbar_try_wait(smem_u32(&bar), 0))
+        wait_slow(smem_u32(&bar), 0, &abort_flag, status, limit_ns, limit_ns);
 }
 
 // ---------------------------------------------------------------- exp2 on the FMA pipe
@@ -339,6 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         o[4 * m + 2] = __float_as_uint(__uint_as_float(o[4 * m + 2]) * alpha_b);
                         o[4 * m + 3] = __float_as_uint(__uint_as_float(o[4 * m + 3]) * alpha_b);
                     }
+                    reg_fence64(o);
                     tmem_st16x256b_x16(t_o, o);
                 } else {
                     uint32_t o[32];
@@ -352,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         o[4 * m + 2] = __float_as_uint(__uint_as_float(o[4 * m + 2]) * alpha_b);
                         o[4 * m + 3] = __float_as_uint(__uint_as_float(o[4 * m + 3]) * alpha_b);
                     }
+                    reg_fence32(o);
                     tmem_st16x256b_x8(t_o, o);
                 }
             }
@@ -363,7 +401,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 2m / 2m+1 = keys 8m + kq + {0,1} of row a / row b, which is the
             // 16x128b store layout at column 4m + t%4 of the P region.
             uint64_t la2 = 0, lb2 = 0, ha2 = 0, hb2 = 0;
+            float hsa0 = 0.f, hsa1 = 0.f, hsb0 = 0.f, hsb1 = 0.f;
             uint32_t pk[32];
+            if constexpr (FA_SOFTMAX_PHASED) {
+                // pass 1: exponents c*s - m, in place
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int m = i >> 1;
+                    const int o = 4 * m + 2 * (i & 1);
+                    const uint64_t x2 = fma2(f2(__uint_as_float(s[o]), __uint_as_float(s[o + 1])), c2,
+                                             (i & 1) ? negb : nega);
+                    float x0, x1;
+                    f2_split(x2, x0, x1);
+                    s[o] = __float_as_uint(x0);
+                    s[o + 1] = __float_as_uint(x1);
+                }
+                // pass 2: exponentials in place
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int o = 4 * (i >> 1) + 2 * (i & 1);
+                    float p0, p1;
+                    if (kEmuEvery > 0 && (i % kEmuEvery) == kEmuEvery - 1) {
+                        exp2_poly2(__uint_as_float(s[o]), __uint_as_float(s[o + 1]), p0, p1);
+                    } else {
+                        p0 = ex2_approx(__uint_as_float(s[o]));
+                        p1 = ex2_approx(__uint_as_float(s[o + 1]));
+                    }
+                    s[o] = __float_as_uint(p0);
+                    s[o + 1] = __float_as_uint(p1);
+                }
+                // pass 3: bf16 pairs and the two sums
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int o = 4 * (i >> 1) + 2 * (i & 1);
+                    const float p0 = __uint_as_float(s[o]), p1 = __uint_as_float(s[o + 1]);
+                    const uint32_t w = pack_bf16x2(p0, p1);
+                    const uint64_t pr = f2(p0, p1);
+                    const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+                    if (i & 1) {
+                        lb2 = add2(lb2, pr);
+                        hb2 = add2(hb2, ph);
+                    } else {
+                        la2 = add2(la2, pr);
+                        ha2 = add2(ha2, ph);
+                    }
+                    pk[i] = w;
+                }
+            } else
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const int m = i >> 1;
@@ -382,16 +466,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint32_t w = pack_bf16x2(p0, p1);
                 const uint64_t pr = f2(p0, p1);
-                const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-                if (row_b) {
-                    lb2 = add2(lb2, pr);
-                    hb2 = add2(hb2, ph);
+                if (row_b) lb2 = add2(lb2, pr);
+                else la2 = add2(la2, pr);
+                if constexpr (FA_LHAT_MIXED_ADD) {
+                    if (row_b) add_bf16x2_halves(hsb0, hsb1, w);
+                    else add_bf16x2_halves(hsa0, hsa1, w);
                 } else {
-                    la2 = add2(la2, pr);
-                    ha2 = add2(ha2, ph);
+                    const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+                    if (row_b) hb2 = add2(hb2, ph);
+                    else ha2 = add2(ha2, ph);
                 }
                 pk[i] = w;
             }
+            // Pin the packed words in registers ahead of the asynchronous
+            // TMEM store.  Without this fence the multi-pass form above was
+            // observed on sm_100a to store stale register contents (the score
+            // tile) instead of P; the fence emits no instruction.
+            reg_fence32(pk);
             tmem_st16x128b_x16(t_s + C::kColP, pk);
             float u0, u1;
             f2_split(la2, u0, u1);
@@ -402,6 +493,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             lh_a += u0 + u1;
             f2_split(hb2, u0, u1);
             lh_b += u0 + u1;
+            lh_a += hsa0 + hsa1;
+            lh_b += hsb0 + hsb1;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p_full + 8 * bb);

@@ -372,6 +372,14 @@ __device__ __forceinline__ uint64_t add2_rm(uint64_t a, uint64_t b) {
     asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+// acc_lo += bf16 low half of w, acc_hi += bf16 high half (fp32 accumulators).
+__device__ __forceinline__ void add_bf16x2_halves(float& acc_lo, float& acc_hi, uint32_t w) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(acc_lo), "+f"(acc_hi)
+        : "r"(w));
+}
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

@@ -104,6 +104,22 @@ int fa_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, fl
                 void* q_d, void* k_d, void* v_d, void* o_d, float* lse_d, int64_t B, int64_t H,
                 int64_t N, int64_t d, int causal, float scale, void* stream);
 
+/*
+ * fa_selftest_wait_timeout - exercises the device-side failure path.
+ *
+ * Launches one small kernel that waits, with the same bounded-wait routine
+ * the attention kernel uses for every pipeline wait, on an mbarrier that
+ * nothing arrives at.  The wait gives up after `limit_us` microseconds and
+ * writes FA_ERR_TIMEOUT into the caller-owned device int `dev_status`; the
+ * kernel then exits normally and the CUDA context stays usable.  With
+ * `arrive` nonzero the barrier is completed first and `dev_status` is left
+ * untouched (the control case).  Nothing faults, traps or hangs.
+ *
+ *   dev_status  device int, caller-owned, not cleared by the call (NULL -> FA_ERR_NULL)
+ *   limit_us    1 .. 10,000,000 (else FA_ERR_SHAPE)
+ */
+int fa_selftest_wait_timeout(int* dev_status, int64_t limit_us, int arrive, void* stream);
+
 /* Number of kernel launches one fa_fwd call makes for these sizes (0 or 1). */
 int fa_fwd_launches(int64_t B, int64_t H, int64_t N, int64_t d);
 

@@ -90,6 +90,12 @@ def test_host_entry_checks():
     assert f(*args, 1, 1, 0, 64, 0, 0.125, None) == fa.FA_OK
 
 
+def test_selftest_argument_checks():
+    assert LIB.fa_selftest_wait_timeout(None, 1000, 0, None) == fa.FA_ERR_NULL
+    assert LIB.fa_selftest_wait_timeout(16, 0, 0, None) == fa.FA_ERR_SHAPE
+    assert LIB.fa_selftest_wait_timeout(16, 10**8, 0, None) == fa.FA_ERR_SHAPE
+
+
 def test_launch_count():
     assert fa.launches_per_call(1, 1, 128, 64) == 1
     assert fa.launches_per_call(0, 1, 128, 64) == 0
