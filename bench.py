@@ -23,9 +23,11 @@ workload with no data-path collective (weak scaling).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -64,6 +66,27 @@ def load_peaks():
                     hbm=float(p["hbm_gbs"]), source="measured")
     except Exception:
         return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+def measured_traffic(workload):
+    """DRAM bytes per non-causal launch from the committed ncu summary, or None
+    when the kernel source changed since the counters were taken (or the
+    summary does not cover this workload)."""
+    if workload != DEFAULT_WORKLOAD:
+        return None, None
+    prof = os.path.join(ROOT, "profiles", "fa_fwd_kernel_b1_h64_n4096_d128_ncu.md")
+    src = os.path.join(ROOT, "attention_forward_17_b200", "csrc", "fa_fwd_kernel.cuh")
+    try:
+        text = open(prof).read()
+        want = re.search(r"kernel_source_sha256_16: (\w+)", text).group(1)
+        have = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if want != have:
+            return None, "kernel changed since the ncu capture"
+        val = float(re.search(r"traffic_bytes_per_launch_noncausal: ([0-9.e+]+)", text).group(1))
+        return val, ("ncu dram__bytes_read+write of one launch at B=1,H=64,N=4096,d=128, scaled x2 by "
+                     "BH*N*d to the workload (profiles/fa_fwd_kernel_b1_h64_n4096_d128_ncu.md)")
+    except (OSError, AttributeError, ValueError):
+        return None, None
 
 
 # ------------------------------------------------------------------ clocks
@@ -185,6 +208,17 @@ def dist_setup(n_gpus):
     return world, rank, local
 
 
+def max_over_ranks(x, world, device=None):
+    """Largest value of x over all ranks (the job's time is its slowest rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_reference(args, cfg):
     """The oracle arm: fp64 CPU attention on bounded row samples per step."""
     world, rank, _ = dist_setup(args.gpus)
@@ -271,13 +305,6 @@ def run_ours(args, cfg):
             import torch.distributed as dist
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        import torch.distributed as dist
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # ---------------- device-resident timing, per-launch events
     for _ in range(args.warmup):
@@ -300,7 +327,7 @@ def run_ours(args, cfg):
         t_end.record(stream)
         torch.cuda.synchronize()
         barrier()
-    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     launch_ms = {c: statistics.mean(a.elapsed_time(b) for a, b in ev[c]) for c in modes}
     clocks = clk.summary()
     value = world * f_step * args.steps / (elapsed_ms / 1e3) / 1e12
@@ -330,7 +357,7 @@ def run_ours(args, cfg):
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = max_over_ranks(a.elapsed_time(b))
+        e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
         tensor_bytes = B * H * N * d * 2
         e2e = {"value": world * f_step * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": 2 * 3 * tensor_bytes,
@@ -341,10 +368,12 @@ def run_ours(args, cfg):
     peaks = load_peaks()
     ach = {c: flops(B, H, N, d, c) / (launch_ms[c] / 1e3) / 1e12 for c in modes}
     dominant = max(modes, key=lambda c: launch_ms[c])
+    traffic, traffic_src = measured_traffic(args.workload)
     roofline = {"bound": "tensor", "kernel": f"fa_fwd_kernel<{d},{str(dominant).lower()}>",
                 "achieved": ach[dominant], "peak": peaks["bf16"], "unit": "TFLOP/s",
                 "frac": ach[dominant] / peaks["bf16"], "peak_source": peaks["source"] + " burst",
-                "traffic": None,
+                "traffic": traffic if dominant is False else None, "traffic_source": traffic_src,
+                "algorithmic_bytes_per_launch": 8.0 * B * H * N * d + 4.0 * B * H * N,
                 "per_mode": {("causal" if c else "non_causal"): {
                     "ms_per_launch": launch_ms[c], "tflops": ach[c],
                     "frac_of_measured_burst": ach[c] / peaks["bf16"],
