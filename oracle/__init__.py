@@ -10,7 +10,8 @@ seeded input generator in ``seeded_inputs``.
   P = row softmax of S,  O = P V,  LSE_i = ln sum_j exp(S[i, j])
 as in the FlashAttention section of the TileLang tutorial (fused forward over
 Q/K/V tiles, validated against scaled-dot-product attention, causal and
-non-causal).  Every function here is pinned by ``tests/test_oracle.py``.
+non-causal).  ``row_softmax`` is the tutorial's row-wise softmax.  Every
+function here is pinned by ``tests/test_oracle.py``.
 """
 from __future__ import annotations
 
@@ -38,6 +39,9 @@ def _lib():
             ctypes.c_int, ctypes.c_double, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p,
             ctypes.c_void_p, ctypes.c_int]
         lib.oracle_attention_rows.restype = ctypes.c_int
+        lib.oracle_row_softmax.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                           ctypes.c_int64, ctypes.c_double, ctypes.c_int]
+        lib.oracle_row_softmax.restype = ctypes.c_int
         lib.oracle_threads.argtypes = []
         lib.oracle_threads.restype = ctypes.c_int
         _LIB = lib
@@ -83,3 +87,15 @@ def attention_rows(q, k, v, causal: bool, scale: float, rows, threads: int = 0):
     if rc != 0:
         raise RuntimeError(f"oracle_attention_rows failed ({rc})")
     return o, lse
+
+
+def row_softmax(x, scale: float = 1.0, threads: int = 0):
+    """fp64 row-wise softmax of bf16 bits x [rows, cols]: exp(scale*x - max) / sum."""
+    x = _bits(x)
+    rows, cols = x.shape
+    y = np.zeros((rows, cols), dtype=np.float64)
+    rc = _lib().oracle_row_softmax(x.ctypes.data, y.ctypes.data, rows, cols, float(scale),
+                                   int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_row_softmax failed ({rc})")
+    return y

@@ -26,6 +26,10 @@
  *
  * Inputs are bf16 bit patterns (uint16, [B, H, N, d], contiguous), widened
  * exactly to fp64.  Outputs are fp64: O [B, H, N, d] and LSE [B, H, N].
+ *
+ * Also here: the row-wise softmax of the tutorial's softmax section (a row's
+ * maximum and sum reductions, then normalisation):
+ *     y[r, c] = exp(scale * x[r, c] - max_c' scale * x[r, c']) / sum_c' exp(...)
  */
 #include <math.h>
 #include <stdint.h>
@@ -180,4 +184,26 @@ int oracle_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* 
         free(s); free(p); free(qr); free(kh); free(vh);
     }
     return status;
+}
+
+/* Row-wise softmax of bf16 bits x [rows, cols] (fp64).  y: rows x cols fp64.
+ * Returns 0, or -1 on bad arguments. */
+int oracle_row_softmax(const uint16_t* x, double* y, int64_t rows, int64_t cols, double scale,
+                       int threads) {
+    if (!x || !y || rows < 0 || cols <= 0) return -1;
+    set_threads(threads);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* xr = x + r * cols;
+        double* yr = y + r * cols;
+        double m = -INFINITY;
+        for (int64_t c = 0; c < cols; ++c) {
+            const double v = scale * bf16_to_double(xr[c]);
+            if (v > m) m = v;
+        }
+        double l = 0.0;
+        for (int64_t c = 0; c < cols; ++c) l += exp(scale * bf16_to_double(xr[c]) - m);
+        for (int64_t c = 0; c < cols; ++c) yr[c] = exp(scale * bf16_to_double(xr[c]) - m) / l;
+    }
+    return 0;
 }

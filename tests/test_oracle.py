@@ -213,3 +213,45 @@ def test_thread_count_does_not_change_result():
     b = oracle.attention_fwd(q, k, v, False, 0.125, threads=4)
     np.testing.assert_array_equal(a[0], b[0])
     np.testing.assert_array_equal(a[1], b[1])
+
+
+# ---------------------------------------------------------------- row softmax
+def row_bits(rows, cols, seed, sigma=1.0):
+    return si.normal_bf16((rows, cols), seed=seed, tensor_id=7, sigma=sigma)
+
+
+@pytest.mark.parametrize("cols", [1, 3, 8, 100, 1000])
+@pytest.mark.parametrize("scale", [1.0, 0.3])
+def test_row_softmax_brute_force(cols, scale):
+    x = row_bits(5, cols, seed=cols)
+    y = oracle.row_softmax(x, scale)
+    xf = f64(x)
+    for r in range(5):
+        lse = math.log(math.fsum(math.exp(scale * v) for v in xf[r]))
+        ref = [math.exp(scale * v - lse) for v in xf[r]]
+        np.testing.assert_allclose(y[r], ref, rtol=1e-12, atol=0)
+
+
+def test_row_softmax_against_torch():
+    x = row_bits(64, 777, seed=1, sigma=4.0)
+    y = oracle.row_softmax(x, 0.7)
+    ref = torch.softmax(0.7 * torch.from_numpy(f64(x)), dim=-1).numpy()
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-300)
+
+
+def test_row_softmax_invariants():
+    x = row_bits(16, 513, seed=2, sigma=3.0)
+    y = oracle.row_softmax(x)
+    np.testing.assert_allclose(y.sum(axis=1), 1.0, rtol=0, atol=1e-12)      # rows sum to one
+    # shift invariance: integer-valued rows plus 16 stay exact in bf16 and give the same softmax
+    xi = np.random.default_rng(4).integers(-20, 20, size=(8, 300)).astype(np.float64)
+    np.testing.assert_allclose(oracle.row_softmax(bits(xi + 16.0)), oracle.row_softmax(bits(xi)),
+                               rtol=1e-14, atol=0)
+    xs = bits(np.full((2, 40), 3.0))                                         # equal entries: uniform
+    np.testing.assert_allclose(oracle.row_softmax(xs), 1.0 / 40, rtol=1e-15)
+    xo = bits(np.where(np.arange(50) == 17, 100.0, 0.0)[None])               # one dominant entry
+    yo = oracle.row_softmax(xo)
+    assert abs(yo[0, 17] - 1.0) < 1e-40 + 1e-15 and yo[0, :17].max() < 1e-40
+    # permuting columns permutes the output
+    perm = np.random.default_rng(3).permutation(513)
+    np.testing.assert_allclose(oracle.row_softmax(x[:, perm]), y[:, perm], rtol=1e-14, atol=0)
