@@ -4,9 +4,9 @@ include/fa.h.  This package is the thin Python binding of that library."""
 from ._binding import (FA_ERR_ALIGN, FA_ERR_ARCH, FA_ERR_CUDA, FA_ERR_HEADDIM, FA_ERR_NULL,
                        FA_ERR_SCALE, FA_ERR_SHAPE, FA_ERR_TIMEOUT, FA_OK, FaError, LIB_PATH,
                        fa_fwd, fa_fwd_host, header_functions, launches_per_call, lib,
-                       selftest_wait_timeout, strerror, version)
+                       row_softmax, selftest_wait_timeout, strerror, version)
 
-__all__ = ["fa_fwd", "fa_fwd_host", "selftest_wait_timeout", "FaError", "strerror", "version", "launches_per_call",
+__all__ = ["fa_fwd", "fa_fwd_host", "row_softmax", "selftest_wait_timeout", "FaError", "strerror", "version", "launches_per_call",
            "header_functions", "lib", "LIB_PATH", "FA_OK", "FA_ERR_NULL", "FA_ERR_SHAPE",
            "FA_ERR_HEADDIM", "FA_ERR_ALIGN", "FA_ERR_SCALE", "FA_ERR_CUDA", "FA_ERR_TIMEOUT",
            "FA_ERR_ARCH"]

@@ -54,6 +54,10 @@ def _load():
     lib.fa_fwd_host.restype = ctypes.c_int
     lib.fa_selftest_wait_timeout.argtypes = [_vp, _i64, ctypes.c_int, _vp]
     lib.fa_selftest_wait_timeout.restype = ctypes.c_int
+    lib.fa_row_softmax.argtypes = [_vp, _vp, _i64, _i64, ctypes.c_float, _vp]
+    lib.fa_row_softmax.restype = ctypes.c_int
+    lib.fa_row_softmax_launches.argtypes = [_i64, _i64]
+    lib.fa_row_softmax_launches.restype = ctypes.c_int
     lib.fa_fwd_launches.argtypes = [_i64, _i64, _i64, _i64]
     lib.fa_fwd_launches.restype = ctypes.c_int
     lib.fa_strerror.argtypes = [ctypes.c_int]
@@ -175,3 +179,24 @@ def selftest_wait_timeout(status, limit_us: int, arrive: bool = False, stream=No
         rc = lib.fa_selftest_wait_timeout(status.data_ptr(), int(limit_us), int(bool(arrive)), s)
     if rc != FA_OK:
         raise FaError(rc, "fa_selftest_wait_timeout")
+
+
+def row_softmax(x, scale: float = 1.0, out=None, stream=None):
+    """y = softmax(scale * x) over the last dimension of a contiguous bf16 CUDA tensor."""
+    import torch
+    if not isinstance(x, torch.Tensor) or x.dtype != torch.bfloat16 or x.device.type != "cuda":
+        raise TypeError("x must be a bfloat16 CUDA tensor")
+    if not x.is_contiguous() or x.dim() < 1:
+        raise ValueError("x must be contiguous with at least one dimension")
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    if out is None:
+        out = torch.empty_like(x)
+    if out.shape != x.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like x")
+    s = (stream if stream is not None else torch.cuda.current_stream(x.device)).cuda_stream
+    with torch.cuda.device(x.device):
+        rc = lib.fa_row_softmax(x.data_ptr(), out.data_ptr(), rows, cols, float(scale), s)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_row_softmax")
+    return out

@@ -27,11 +27,11 @@ def library_path() -> str:
 
 
 def _sources():
-    return [os.path.join(CSRC, "fa_fwd.cu")]
+    return [os.path.join(CSRC, "fa_fwd.cu"), os.path.join(CSRC, "row_softmax.cu")]
 
 
 def _deps():
-    return (glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+    return (_sources() + glob.glob(os.path.join(CSRC, "*.cuh"))
             + glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 

@@ -409,12 +409,63 @@ def run_ours(args, cfg):
         dist.destroy_process_group()
 
 
+def bench_row_softmax(args):
+    """One JSON line for the row-wise softmax kernel (HBM-bound)."""
+    import numpy as np
+    import torch
+    import attention_forward_17_b200 as fa
+    import seeded_inputs as si
+    rows, cols = 32768, 4096
+    bits = si.normal_bf16((rows, cols), seed=0, tensor_id=7, sigma=2.0)
+    x = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    y = torch.empty_like(x)
+    for _ in range(args.warmup):
+        fa.row_softmax(x, 1.0, out=y)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # inputs + outputs (512 MiB) exceed L2, so consecutive launches re-read HBM
+    with ClockSampler(0) as clk:
+        a.record()
+        for _ in range(args.steps):
+            fa.row_softmax(x, 1.0, out=y)
+        b.record()
+        torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    nbytes = 2.0 * 2 * rows * cols
+    gbs = nbytes / (ms / 1e3) / 1e9
+    peaks = load_peaks()
+    # CPU baseline: the oracle on a sample of rows
+    import oracle
+    t0 = time.perf_counter()
+    sample = 512
+    ref = oracle.row_softmax(bits[:sample], 1.0)
+    dt = time.perf_counter() - t0
+    got = y[:sample].float().cpu().numpy().astype(np.float64)
+    worst = float(np.max(np.abs(got - ref) / (np.abs(ref) + 1e-30)))
+    line = {"metric": "row softmax GB/s (bf16 in, bf16 out)", "value": gbs, "unit": "GB/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": f"row_softmax_r{rows}_c{cols}", "rows": rows,
+                                            "cols": cols, "l2": "512 MiB moved per launch, above L2"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm"], "traffic": None,
+                         "algorithmic_bytes_per_launch": nbytes},
+            "cpu_baseline": {"value": sample * cols * 4 / dt / 1e9, "unit": "GB/s",
+                             "cores": oracle.default_threads(), "kind": "oracle",
+                             "sample": f"{sample} rows", "max_rel_err_vs_gpu": worst},
+            "gpu_launches": args.steps * fa.lib.fa_row_softmax_launches(rows, cols),
+            "clocks": clk.summary(), "impl": "ours"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--suite", choices=["attention", "next"], default="attention",
+                    help="'next' measures the kernels beyond the attention path, one line each")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--modes", choices=sorted(MODES), default="both",
                     help="masking modes in one step (the headline uses both)")
@@ -428,6 +479,9 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     cfg = WORKLOADS[args.workload]
+    if args.suite == "next":
+        bench_row_softmax(args)
+        return
     if args.impl == "reference":
         run_reference(args, cfg)
     else:

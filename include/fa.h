@@ -120,6 +120,27 @@ int fa_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, fl
  */
 int fa_selftest_wait_timeout(int* dev_status, int64_t limit_us, int arrive, void* stream);
 
+/*
+ * fa_row_softmax - row-wise softmax (the tutorial's softmax section: fragment
+ * maximum and sum reductions, normalisation kept in registers).
+ *
+ *     y[r, c] = exp(scale * x[r, c] - max_c' scale * x[r, c']) / sum_c' exp(...)
+ *
+ *   x      device, bf16 [rows, cols], dense row-major, finite values, read only.
+ *   y      device, bf16 [rows, cols], written (may not overlap x unless equal to it).
+ *   rows   0 .. 2^31 - 1; cols 0 .. 2^31 - 1 (a zero is a no-op returning FA_OK).
+ *   scale  any finite value (FA_ERR_SCALE otherwise).
+ * x and y must be 2-byte aligned (FA_ERR_ALIGN).  fp32 arithmetic, output
+ * rounded to nearest even.  Rows with cols % 8 == 0, 16-byte aligned
+ * pointers and cols <= 16384 are read once and written once; other shapes
+ * read the row twice.  Asynchronous on `stream`; FA_ERR_ARCH on a non-sm_100
+ * device; nothing is allocated.
+ */
+int fa_row_softmax(const void* x, void* y, int64_t rows, int64_t cols, float scale, void* stream);
+
+/* Number of kernel launches one fa_row_softmax call makes (0 or 1). */
+int fa_row_softmax_launches(int64_t rows, int64_t cols);
+
 /* Number of kernel launches one fa_fwd call makes for these sizes (0 or 1). */
 int fa_fwd_launches(int64_t B, int64_t H, int64_t N, int64_t d);
 

@@ -96,6 +96,17 @@ def test_selftest_argument_checks():
     assert LIB.fa_selftest_wait_timeout(16, 10**8, 0, None) == fa.FA_ERR_SHAPE
 
 
+def test_row_softmax_argument_checks():
+    f = LIB.fa_row_softmax
+    assert f(16, 32, -1, 8, 1.0, None) == fa.FA_ERR_SHAPE
+    assert f(0, 0, 0, 8, 1.0, None) == fa.FA_OK
+    assert f(0, 32, 4, 8, 1.0, None) == fa.FA_ERR_NULL
+    assert f(17, 32, 4, 8, 1.0, None) == fa.FA_ERR_ALIGN
+    assert f(16, 32, 4, 8, float("inf"), None) == fa.FA_ERR_SCALE
+    assert f(16, 32, 2 ** 31, 8, 1.0, None) == fa.FA_ERR_SHAPE
+    assert LIB.fa_row_softmax_launches(4, 8) == 1 and LIB.fa_row_softmax_launches(0, 8) == 0
+
+
 def test_launch_count():
     assert fa.launches_per_call(1, 1, 128, 64) == 1
     assert fa.launches_per_call(0, 1, 128, 64) == 0
