@@ -10,8 +10,10 @@ seeded input generator in ``seeded_inputs``.
   P = row softmax of S,  O = P V,  LSE_i = ln sum_j exp(S[i, j])
 as in the FlashAttention section of the TileLang tutorial (fused forward over
 Q/K/V tiles, validated against scaled-dot-product attention, causal and
-non-causal).  ``row_softmax`` is the tutorial's row-wise softmax.  Every
-function here is pinned by ``tests/test_oracle.py``.
+non-causal).  ``row_softmax`` is the tutorial's row-wise softmax, ``gemm`` its
+tiled matrix multiplication with the optional fused bias / bias + GELU
+epilogue, ``vector_add`` its elementwise addition.  Every function here is
+pinned by ``tests/test_oracle.py`` or ``tests/test_oracle_gemm.py``.
 """
 from __future__ import annotations
 
@@ -42,6 +44,14 @@ def _lib():
         lib.oracle_row_softmax.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                            ctypes.c_int64, ctypes.c_double, ctypes.c_int]
         lib.oracle_row_softmax.restype = ctypes.c_int
+        lib.oracle_gemm.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64] * 3 + [
+            ctypes.c_int, ctypes.c_int]
+        lib.oracle_gemm.restype = ctypes.c_int
+        lib.oracle_gemm_entries.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 3 + [
+            ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int]
+        lib.oracle_gemm_entries.restype = ctypes.c_int
+        lib.oracle_vector_add.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64, ctypes.c_int]
+        lib.oracle_vector_add.restype = ctypes.c_int
         lib.oracle_threads.argtypes = []
         lib.oracle_threads.restype = ctypes.c_int
         _LIB = lib
@@ -99,3 +109,55 @@ def row_softmax(x, scale: float = 1.0, threads: int = 0):
     if rc != 0:
         raise RuntimeError(f"oracle_row_softmax failed ({rc})")
     return y
+
+
+GEMM_PLAIN, GEMM_BIAS, GEMM_BIAS_GELU = 0, 1, 2
+
+
+def _ptr(a):
+    return a.ctypes.data if a is not None and a.size else None
+
+
+def gemm(a, b, bias=None, mode: int = GEMM_BIAS_GELU, threads: int = 0):
+    """fp64 C [M, N] = epilogue(A B) for bf16 bits A [M, K], B [K, N], bias [N]."""
+    a, b = _bits(a), _bits(b)
+    M, K = a.shape
+    K2, N = b.shape
+    assert K == K2
+    bias = None if bias is None else _bits(bias)
+    if mode and bias is not None:
+        assert bias.shape == (N,)
+    c = np.zeros((M, N), dtype=np.float64)
+    rc = _lib().oracle_gemm(_ptr(a), _ptr(b), _ptr(bias), c.ctypes.data, M, N, K, int(mode),
+                            int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_gemm failed ({rc})")
+    return c
+
+
+def gemm_entries(a, b, bias, idx, mode: int = GEMM_BIAS_GELU, threads: int = 0):
+    """C entries at flat indices idx (i * N + j), arithmetic as ``gemm``."""
+    a, b = _bits(a), _bits(b)
+    M, K = a.shape
+    N = b.shape[1]
+    bias = None if bias is None else _bits(bias)
+    r = np.ascontiguousarray(np.asarray(idx, dtype=np.int64))
+    out = np.zeros(len(r), dtype=np.float64)
+    rc = _lib().oracle_gemm_entries(_ptr(a), _ptr(b), _ptr(bias), M, N, K, int(mode),
+                                    r.ctypes.data, len(r), out.ctypes.data, int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_gemm_entries failed ({rc})")
+    return out
+
+
+def vector_add(x, y, threads: int = 0):
+    """fp64 z = x + y for float32 x, y of equal length."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    assert x.shape == y.shape
+    z = np.zeros(x.shape, dtype=np.float64)
+    rc = _lib().oracle_vector_add(x.ctypes.data, y.ctypes.data, z.ctypes.data, x.size,
+                                  int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_vector_add failed ({rc})")
+    return z

@@ -8,6 +8,7 @@ import os
 import subprocess
 
 HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCES = ["attention_oracle.c", "gemm_oracle.c", "vector_add_oracle.c"]
 
 
 def library_path() -> str:
@@ -15,14 +16,15 @@ def library_path() -> str:
 
 
 def build(force: bool = False) -> str:
-    src = os.path.join(HERE, "attention_oracle.c")
+    srcs = [os.path.join(HERE, f) for f in SOURCES]
     out = library_path()
-    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+    if not force and os.path.exists(out) and all(
+            os.path.getmtime(out) >= os.path.getmtime(s) for s in srcs):
         return out
     tmp = out + ".tmp"
     # -O2 without -ffast-math: IEEE fp64, sums taken in the written order.
     subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c11",
-                           "-fno-fast-math", "-ffp-contract=off", src, "-o", tmp, "-lm"])
+                           "-fno-fast-math", "-ffp-contract=off", *srcs, "-o", tmp, "-lm"])
     os.replace(tmp, out)
     return out
 

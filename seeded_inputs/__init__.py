@@ -1,11 +1,12 @@
-"""Seeded synthetic bf16 inputs shared by the oracle and the CUDA path.
+"""Seeded synthetic inputs shared by the oracle and the CUDA path.
 
 The generator (Philox4x32-10 counter-based bits, Box-Muller normals, one
 round-to-nearest-even step to bf16) lives in ``philox_normal.c``; this module
-only builds and calls it.  It holds none of the attention arithmetic, so
+only builds and calls it.  It holds none of the kernels' arithmetic, so
 importing it from both sides couples nothing but the input bytes.
 
-Tensors are returned as numpy ``uint16`` arrays of bf16 bit patterns.
+bf16 tensors are returned as numpy ``uint16`` arrays of bit patterns, fp32
+tensors as ``float32`` arrays.
 """
 from __future__ import annotations
 
@@ -19,6 +20,8 @@ from .build import build as _build, library_path
 _LIB = None
 
 TENSOR_Q, TENSOR_K, TENSOR_V = 0, 1, 2
+TENSOR_GEMM_A, TENSOR_GEMM_B, TENSOR_GEMM_BIAS = 3, 4, 5
+TENSOR_ADD_X, TENSOR_ADD_Y = 6, 7
 
 
 def _lib():
@@ -31,6 +34,9 @@ def _lib():
         lib.seeded_normal_bf16.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64,
                                            ctypes.c_uint32, ctypes.c_double]
         lib.seeded_normal_bf16.restype = None
+        lib.seeded_normal_f32.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64,
+                                          ctypes.c_uint32, ctypes.c_double]
+        lib.seeded_normal_f32.restype = None
         lib.seeded_philox4x32.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                           ctypes.c_void_p]
         lib.seeded_philox4x32.restype = None
@@ -62,6 +68,32 @@ def normal_bf16(shape, seed: int, tensor_id: int, sigma: float = 1.0) -> np.ndar
         _lib().seeded_normal_bf16(out.ctypes.data, n, int(seed) & (2**64 - 1),
                                   int(tensor_id), float(sigma))
     return out.reshape(shape)
+
+
+def normal_f32(shape, seed: int, tensor_id: int, sigma: float = 1.0) -> np.ndarray:
+    """float32 iid N(0, sigma^2): the draws of ``normal_bf16`` rounded to fp32 instead."""
+    n = int(np.prod(shape)) if len(shape) else 1
+    out = np.empty(n, dtype=np.float32)
+    if n:
+        _lib().seeded_normal_f32(out.ctypes.data, n, int(seed) & (2**64 - 1), int(tensor_id),
+                                 float(sigma))
+    return out.reshape(shape)
+
+
+def make_gemm(M: int, N: int, K: int, seed: int = 0):
+    """A [M, K], B [K, N], bias [N] as bf16 bits: A ~ N(0, 1), B ~ N(0, 1/K), bias ~ N(0, 1).
+
+    B's scale keeps the pre-activation A B + bias near unit variance, so the
+    GELU epilogue acts on values where it is far from linear."""
+    a = normal_bf16((M, K), seed, TENSOR_GEMM_A, 1.0)
+    b = normal_bf16((K, N), seed, TENSOR_GEMM_B, 1.0 / max(K, 1) ** 0.5)
+    bias = normal_bf16((N,), seed, TENSOR_GEMM_BIAS, 1.0)
+    return a, b, bias
+
+
+def make_add(n: int, seed: int = 0):
+    """x, y float32 [n], iid N(0, 1)."""
+    return normal_f32((n,), seed, TENSOR_ADD_X), normal_f32((n,), seed, TENSOR_ADD_Y)
 
 
 def make_qkv(B: int, H: int, N: int, d: int, seed: int = 0, sigma_qk: float = 1.0,

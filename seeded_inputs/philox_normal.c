@@ -1,8 +1,9 @@
 /*
- * Seeded synthetic inputs for the attention forward pass: bf16 tensors whose
- * elements are independent N(0, sigma^2) draws.
+ * Seeded synthetic inputs for the attention forward pass and the other kernels
+ * of the library: bf16 (or fp32) tensors whose elements are independent
+ * N(0, sigma^2) draws.
  *
- * This module holds no attention arithmetic.  Both the fp64 oracle and the
+ * This module holds none of the kernels' arithmetic.  Both the fp64 oracle and the
  * CUDA path read the bytes it writes, so the two see identical inputs.
  *
  * Generator, stated from its published definitions:
@@ -22,7 +23,8 @@
  *   - value = sigma * z (double), rounded once, to nearest-even, to bf16.
  *
  * The tensor is written as raw bf16 bit patterns (uint16), row-major, in the
- * order of the flat element index.
+ * order of the flat element index.  seeded_normal_f32 writes the same draws
+ * rounded once (nearest-even) to fp32 instead.
  */
 #include <math.h>
 #include <stdint.h>
@@ -77,27 +79,47 @@ uint16_t seeded_round_bf16(double x) {
     return (uint16_t)(bits >> 16);
 }
 
-/* Fill out[0 .. n) with bf16(sigma * N(0,1)) for (seed, tensor_id). */
-void seeded_normal_bf16(uint16_t* out, int64_t n, uint64_t seed, uint32_t tensor_id,
-                        double sigma) {
+/* The four N(0,1) draws of Philox call c for (seed, tensor_id). */
+static void normal4(uint64_t seed, uint32_t tensor_id, int64_t c, double z[4]) {
     const double two_pi = 6.283185307179586476925286766559;
     const double inv_2_32 = 1.0 / 4294967296.0;
     uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32) ^ tensor_id};
+    uint32_t ctr[4] = {(uint32_t)c, (uint32_t)((uint64_t)c >> 32), 0u, 0u};
+    uint32_t w[4];
+    seeded_philox4x32(ctr, key, 10, w);
+    for (int p = 0; p < 2; ++p) {
+        double u0 = ((double)w[2 * p] + 0.5) * inv_2_32;
+        double u1 = ((double)w[2 * p + 1] + 0.5) * inv_2_32;
+        double r = sqrt(-2.0 * log(u0));
+        double t = two_pi * u1;
+        z[2 * p] = r * cos(t);
+        z[2 * p + 1] = r * sin(t);
+    }
+}
+
+/* Fill out[0 .. n) with fp32(sigma * N(0,1)) for (seed, tensor_id); the same
+ * draws as seeded_normal_bf16, rounded to fp32 instead of bf16. */
+void seeded_normal_f32(float* out, int64_t n, uint64_t seed, uint32_t tensor_id, double sigma) {
     int64_t ncalls = (n + 3) / 4;
 #pragma omp parallel for schedule(static)
     for (int64_t c = 0; c < ncalls; ++c) {
-        uint32_t ctr[4] = {(uint32_t)c, (uint32_t)((uint64_t)c >> 32), 0u, 0u};
-        uint32_t w[4];
-        seeded_philox4x32(ctr, key, 10, w);
         double z[4];
-        for (int p = 0; p < 2; ++p) {
-            double u0 = ((double)w[2 * p] + 0.5) * inv_2_32;
-            double u1 = ((double)w[2 * p + 1] + 0.5) * inv_2_32;
-            double r = sqrt(-2.0 * log(u0));
-            double t = two_pi * u1;
-            z[2 * p] = r * cos(t);
-            z[2 * p + 1] = r * sin(t);
+        normal4(seed, tensor_id, c, z);
+        for (int i = 0; i < 4; ++i) {
+            int64_t idx = 4 * c + i;
+            if (idx < n) out[idx] = (float)(sigma * z[i]);
         }
+    }
+}
+
+/* Fill out[0 .. n) with bf16(sigma * N(0,1)) for (seed, tensor_id). */
+void seeded_normal_bf16(uint16_t* out, int64_t n, uint64_t seed, uint32_t tensor_id,
+                        double sigma) {
+    int64_t ncalls = (n + 3) / 4;
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < ncalls; ++c) {
+        double z[4];
+        normal4(seed, tensor_id, c, z);
         for (int i = 0; i < 4; ++i) {
             int64_t idx = 4 * c + i;
             if (idx < n) out[idx] = seeded_round_bf16(sigma * z[i]);

@@ -79,3 +79,19 @@ def test_values_are_bf16_of_sigma_z():
     f = si.bf16_bits_to_f32(bits)
     again = np.array([si.round_bf16(float(t)) for t in f], dtype=np.uint16)
     assert np.array_equal(bits, again)
+
+
+def test_f32_stream_is_the_bf16_stream_unrounded():
+    # the fp32 and bf16 tensors of one (seed, tensor) come from the same draws
+    x = si.normal_f32((200_000,), seed=5, tensor_id=6)
+    b = si.bf16_bits_to_f32(si.normal_bf16((200_000,), seed=5, tensor_id=6))
+    assert np.all(np.abs(b - x) <= 2.0 ** -8 * np.abs(x) + 1e-30)
+    x_b = torch.as_tensor(x).to(torch.bfloat16).float().numpy()
+    # rounding the fp32 value to bf16 differs from the direct rounding only at double-rounding ties
+    assert (x_b == b).mean() > 0.999
+
+
+def test_gemm_inputs_scale():
+    a, b, bias = si.make_gemm(64, 64, 256, seed=0)
+    assert a.shape == (64, 256) and b.shape == (256, 64) and bias.shape == (64,)
+    assert abs(si.bf16_bits_to_f32(b).std() * 16 - 1) < 0.05
