@@ -1,7 +1,8 @@
 """ctypes binding of libfa_b200.so (include/fa.h).
 
-Argument marshalling only: every step of the attention forward pass runs in
-the library's CUDA kernels.  PyTorch supplies device memory and the current
+Argument marshalling only: every step of the attention forward pass (and of
+the row softmax, GEMM and vector-add entry points) runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current
 stream.  There is no fallback: if the library is missing or the device is not
 sm_100, calls raise.
 """
@@ -26,6 +27,9 @@ FA_ERR_SCALE = -5
 FA_ERR_CUDA = -6
 FA_ERR_TIMEOUT = -7
 FA_ERR_ARCH = -8
+FA_ERR_ARG = -9
+
+FA_GEMM_PLAIN, FA_GEMM_BIAS, FA_GEMM_BIAS_GELU = 0, 1, 2
 
 _i64 = ctypes.c_int64
 _vp = ctypes.c_void_p
@@ -58,6 +62,14 @@ def _load():
     lib.fa_row_softmax.restype = ctypes.c_int
     lib.fa_row_softmax_launches.argtypes = [_i64, _i64]
     lib.fa_row_softmax_launches.restype = ctypes.c_int
+    lib.fa_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp]
+    lib.fa_gemm.restype = ctypes.c_int
+    lib.fa_gemm_launches.argtypes = [_i64, _i64, _i64]
+    lib.fa_gemm_launches.restype = ctypes.c_int
+    lib.fa_vector_add.argtypes = [_vp, _vp, _vp, _i64, _vp]
+    lib.fa_vector_add.restype = ctypes.c_int
+    lib.fa_vector_add_launches.argtypes = [_i64]
+    lib.fa_vector_add_launches.restype = ctypes.c_int
     lib.fa_fwd_launches.argtypes = [_i64, _i64, _i64, _i64]
     lib.fa_fwd_launches.restype = ctypes.c_int
     lib.fa_strerror.argtypes = [ctypes.c_int]
@@ -199,4 +211,60 @@ def row_softmax(x, scale: float = 1.0, out=None, stream=None):
         rc = lib.fa_row_softmax(x.data_ptr(), out.data_ptr(), rows, cols, float(scale), s)
     if rc != FA_OK:
         raise FaError(rc, "fa_row_softmax")
+    return out
+
+
+def gemm(a, b, bias=None, epilogue: int = FA_GEMM_BIAS_GELU, out=None, stream=None, status=None):
+    """C = epilogue(A @ B) for contiguous bf16 CUDA tensors A [M, K], B [K, N], bias [N].
+
+    ``epilogue`` is FA_GEMM_PLAIN, FA_GEMM_BIAS or FA_GEMM_BIAS_GELU (exact erf
+    GELU).  ``out`` (bf16 [M, N]) is allocated when not given.  ``status`` may
+    be an int32 CUDA tensor with one element (receives FA_ERR_TIMEOUT).
+    """
+    import torch
+    for name, t in (("a", a), ("b", b)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.device.type != "cuda":
+            raise TypeError(f"{name} must be a bfloat16 CUDA tensor")
+        if t.dim() != 2 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 2-D tensor")
+    M, K = a.shape
+    K2, N = b.shape
+    if K != K2:
+        raise ValueError(f"inner dimensions differ: {tuple(a.shape)} @ {tuple(b.shape)}")
+    if bias is not None and (bias.dtype != torch.bfloat16 or tuple(bias.shape) != (N,)
+                             or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous bf16 [N] tensor")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != (M, N) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 [M, N] tensor")
+    s = (stream if stream is not None else torch.cuda.current_stream(a.device)).cuda_stream
+    with torch.cuda.device(a.device):
+        rc = lib.fa_gemm(a.data_ptr() if K else None, b.data_ptr() if K else None,
+                         bias.data_ptr() if bias is not None else None, out.data_ptr(), M, N, K,
+                         int(epilogue), status.data_ptr() if status is not None else None, s)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_gemm")
+    return out
+
+
+def vector_add(x, y, out=None, stream=None):
+    """z = x + y for contiguous fp32 CUDA tensors of equal shape."""
+    import torch
+    for name, t in (("x", x), ("y", y)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or t.device.type != "cuda":
+            raise TypeError(f"{name} must be a float32 CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if x.shape != y.shape:
+        raise ValueError("x and y shapes differ")
+    if out is None:
+        out = torch.empty_like(x)
+    if out.shape != x.shape or out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous float32 tensor shaped like x")
+    s = (stream if stream is not None else torch.cuda.current_stream(x.device)).cuda_stream
+    with torch.cuda.device(x.device):
+        rc = lib.fa_vector_add(x.data_ptr(), y.data_ptr(), out.data_ptr(), x.numel(), s)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_vector_add")
     return out

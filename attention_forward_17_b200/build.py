@@ -27,11 +27,13 @@ def library_path() -> str:
 
 
 def _sources():
-    return [os.path.join(CSRC, "fa_fwd.cu"), os.path.join(CSRC, "row_softmax.cu")]
+    return [os.path.join(CSRC, f) for f in
+            ("fa_fwd.cu", "row_softmax.cu", "gemm_bias_gelu.cu", "vector_add.cu")]
 
 
 def _deps():
     return (_sources() + glob.glob(os.path.join(CSRC, "*.cuh"))
+            + glob.glob(os.path.join(CSRC, "*.h"))
             + glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 

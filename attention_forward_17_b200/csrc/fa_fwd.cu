@@ -11,6 +11,7 @@
 
 #include "../../include/fa.h"
 #include "fa_fwd_kernel.cuh"
+#include "host_common.h"
 
 namespace {
 
@@ -23,7 +24,6 @@ struct DeviceState {
 DeviceState g_devices[kMaxDevices];
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
 
 // Opts the instantiation into its dynamic shared memory and checks that it was
 // compiled with enough registers for the in-kernel warpgroup rebalance (a
@@ -66,14 +66,7 @@ int current_device_ready() {
 }
 
 int encoder_ready() {
-    std::call_once(g_encode_once, [] {
-        void* fn = nullptr;
-        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    });
+    g_encode = fa::host::tensor_map_encoder();
     return g_encode ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -92,7 +85,7 @@ int encode_qkv_map(CUtensorMap* map, const void* ptr, int64_t BH, int64_t N, int
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+using fa::host::aligned;
 
 constexpr int64_t kMaxN = (int64_t(1) << 31) - 512;
 constexpr int64_t kMaxBH = (int64_t(1) << 31) - 1;
@@ -215,6 +208,7 @@ const char* fa_strerror(int status) {
         case FA_ERR_CUDA: return "a CUDA runtime or driver call failed";
         case FA_ERR_TIMEOUT: return "a device-side pipeline wait ran out of time";
         case FA_ERR_ARCH: return "the current device is not an sm_100 (B200-class) GPU";
+        case FA_ERR_ARG: return "an enumerated argument is out of range";
         default: return "unknown status";
     }
 }

@@ -1,4 +1,4 @@
-// Thin inline-PTX wrappers for the sm_100a features the attention kernel uses:
+// Thin inline-PTX wrappers for the sm_100a features the library's kernels use:
 // mbarriers, TMA tensor loads, tcgen05 (tensor-memory allocation, MMA,
 // commit, loads/stores, fences) and the special-function exp2/log2 units.
 //
@@ -69,6 +69,16 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int 
         ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(bar),
           "l"(cache_policy)
+        : "memory");
+}
+
+// 2-D tiled load into shared memory, completing `bytes` on the mbarrier.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int c0, int c1,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(bar)
         : "memory");
 }
 

@@ -458,6 +458,121 @@ def bench_row_softmax(args):
     print(json.dumps(line), flush=True)
 
 
+def _event_loop(fn, steps):
+    """Mean device time (ms) of `fn` over `steps` back-to-back launches, CUDA
+    events on the current stream, with clocks sampled meanwhile."""
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps, clk.summary()
+
+
+def bench_gemm(args):
+    """One JSON line for the tcgen05 GEMM with the fused bias + GELU epilogue
+    (tensor-bound), with cuBLAS (torch eager) timed beside it for context."""
+    import numpy as np
+    import torch
+    import attention_forward_17_b200 as fa
+    import seeded_inputs as si
+    M = N = K = 8192
+    a_b, b_b, bias_b = si.make_gemm(M, N, K, seed=0)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).cuda()
+    a, b, bias = dev(a_b), dev(b_b), dev(bias_b)
+    c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    run = lambda: fa.gemm(a, b, bias, fa.FA_GEMM_BIAS_GELU, out=c)
+    for _ in range(args.warmup):
+        run()
+    ms, clocks = _event_loop(run, args.steps)
+    flop = 2.0 * M * N * K
+    tf = flop / (ms / 1e3) / 1e12
+    # context: cuBLAS through torch, plain product and the eager three-kernel epilogue
+    eager = lambda: torch.nn.functional.gelu(a @ b + bias)
+    plain = lambda: a @ b
+    for _ in range(args.warmup):
+        eager(); plain()
+    ms_eager, _ = _event_loop(eager, args.steps)
+    ms_plain, _ = _event_loop(plain, args.steps)
+    peaks = load_peaks()
+    import oracle
+    # CPU baseline: the oracle on sampled entries, sized to a few seconds
+    rng = np.random.default_rng(0)
+    n = 512
+    while True:
+        idx = rng.integers(0, M * N, n)
+        t0 = time.perf_counter()
+        ref = oracle.gemm_entries(a_b, b_b, bias_b, idx, 2)
+        dt = time.perf_counter() - t0
+        if dt > 2.0 or n >= 1 << 20:
+            break
+        n *= 4
+    got = c.float().cpu().numpy().reshape(-1)[idx].astype(np.float64)
+    worst = float(np.max(np.abs(got - ref) - 2.0 ** -8 * np.abs(ref)))
+    line = {"metric": "GEMM + bias + GELU TFLOP/s (bf16 in, fp32 accumulate, bf16 out)",
+            "value": tf, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"gemm_bias_gelu_m{M}_n{N}_k{K}", "M": M, "N": N, "K": K,
+                       "l2": "A, B, C = 384 MiB, above L2"},
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16"],
+                         "unit": "TFLOP/s", "frac": tf / peaks["bf16"], "traffic": None,
+                         "algorithmic_flops_per_launch": flop,
+                         "peak_source": peaks["source"] + " bf16 burst (cuBLAS 8192^3)"},
+            "context": {"cublas_plain_tflops": flop / (ms_plain / 1e3) / 1e12,
+                        "torch_eager_gelu_bias_tflops": flop / (ms_eager / 1e3) / 1e12},
+            "cpu_baseline": {"value": len(idx) * 2.0 * K / dt / 1e12, "unit": "TFLOP/s",
+                             "cores": oracle.default_threads(), "kind": "oracle",
+                             "sample": f"{len(idx)} random entries of C",
+                             "max_excess_err_vs_gpu": worst},
+            "gpu_launches": args.steps * fa.lib.fa_gemm_launches(M, N, K),
+            "clocks": clocks, "impl": "ours"}
+    print(json.dumps(line), flush=True)
+
+
+def bench_vector_add(args):
+    """One JSON line for the fp32 vector add (HBM-bound)."""
+    import numpy as np
+    import torch
+    import attention_forward_17_b200 as fa
+    import seeded_inputs as si
+    n = 1 << 28
+    xh, yh = si.make_add(n, seed=0)
+    x, y = torch.from_numpy(xh).cuda(), torch.from_numpy(yh).cuda()
+    z = torch.empty_like(x)
+    run = lambda: fa.vector_add(x, y, out=z)
+    for _ in range(args.warmup):
+        run()
+    ms, clocks = _event_loop(run, args.steps)
+    nbytes = 12.0 * n
+    gbs = nbytes / (ms / 1e3) / 1e9
+    peaks = load_peaks()
+    import oracle
+    m = 1 << 26
+    t0 = time.perf_counter()
+    ref = oracle.vector_add(xh[:m], yh[:m])
+    dt = time.perf_counter() - t0
+    exact = bool(np.array_equal(z[:m].cpu().numpy(), ref.astype(np.float32)))
+    line = {"metric": "vector add GB/s (fp32)", "value": gbs, "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": f"vector_add_n{n}", "n": n,
+                                            "l2": "3 GiB moved per launch, above L2"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm"], "traffic": None,
+                         "algorithmic_bytes_per_launch": nbytes},
+            "cpu_baseline": {"value": m * 12.0 / dt / 1e9, "unit": "GB/s",
+                             "cores": oracle.default_threads(), "kind": "oracle",
+                             "sample": f"first {m} elements", "bit_exact_vs_gpu": exact},
+            "gpu_launches": args.steps * fa.lib.fa_vector_add_launches(n),
+            "clocks": clocks, "impl": "ours"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -466,6 +581,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--suite", choices=["attention", "next"], default="attention",
                     help="'next' measures the kernels beyond the attention path, one line each")
+    ap.add_argument("--next", nargs="+", choices=["row_softmax", "gemm", "vector_add"],
+                    default=["row_softmax", "gemm", "vector_add"],
+                    help="kernels measured by --suite next")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--modes", choices=sorted(MODES), default="both",
                     help="masking modes in one step (the headline uses both)")
@@ -480,7 +598,9 @@ def main():
         raise SystemExit("--warmup must be >= 3")
     cfg = WORKLOADS[args.workload]
     if args.suite == "next":
-        bench_row_softmax(args)
+        for name in args.next:
+            {"row_softmax": bench_row_softmax, "gemm": bench_gemm,
+             "vector_add": bench_vector_add}[name](args)
         return
     if args.impl == "reference":
         run_reference(args, cfg)

@@ -2,7 +2,7 @@
  * fa.h - C ABI of the B200 (sm_100a) fused attention forward library
  * (libfa_b200.so).
  *
- * The operation is the fused FlashAttention forward pass of the "TileLang
+ * The main operation is the fused FlashAttention forward pass of the "TileLang
  * tutorial" (FlashAttention section): query, key and value tiles are processed
  * without materialising the attention-score matrix in global memory, using an
  * online softmax (running row maxima, running normalisation sums, rescaling
@@ -16,6 +16,10 @@
  * alignment; query and key lengths are equal).  The pages validate this
  * against scaled-dot-product attention; LSE is the natural-log logsumexp of the
  * scaled scores.
+ *
+ * The library also carries the tutorial's other kernels, each behind its own
+ * entry point below: the row-wise softmax, the tiled tensor-core GEMM with
+ * its fused bias + GELU epilogue, and the vector addition.
  *
  * Layout: Q, K, V and O are bf16 [B, H, N, d], dense row-major (d fastest), in
  * device memory.  LSE is fp32 [B, H, N].  d must be 64 or 128.  Arithmetic:
@@ -51,7 +55,8 @@ typedef enum {
     FA_ERR_SCALE = -5,    /* scale is not finite and > 0                             */
     FA_ERR_CUDA = -6,     /* a CUDA runtime/driver call failed                       */
     FA_ERR_TIMEOUT = -7,  /* a device-side pipeline wait ran out of time             */
-    FA_ERR_ARCH = -8      /* the current device is not compute capability 10.0       */
+    FA_ERR_ARCH = -8,     /* the current device is not compute capability 10.0       */
+    FA_ERR_ARG = -9       /* an enumerated argument is out of range                  */
 } fa_status;
 
 /*
@@ -140,6 +145,66 @@ int fa_row_softmax(const void* x, void* y, int64_t rows, int64_t cols, float sca
 
 /* Number of kernel launches one fa_row_softmax call makes (0 or 1). */
 int fa_row_softmax_launches(int64_t rows, int64_t cols);
+
+/* Epilogues of fa_gemm. */
+typedef enum {
+    FA_GEMM_PLAIN = 0,     /* C = A B                              */
+    FA_GEMM_BIAS = 1,      /* C = A B + bias                       */
+    FA_GEMM_BIAS_GELU = 2  /* C = GELU(A B + bias), exact erf form */
+} fa_gemm_epilogue;
+
+/*
+ * fa_gemm - tiled tensor-core matrix product with a fused epilogue (the
+ * tutorial's tiled GEMM section, and its fused-epilogue section: bias and
+ * GELU applied to the accumulator before the only store of C).
+ *
+ *     C[i, j] = epi( sum_k A[i, k] B[k, j] )
+ *        FA_GEMM_PLAIN      epi(x) = x
+ *        FA_GEMM_BIAS       epi(x) = x + bias[j]
+ *        FA_GEMM_BIAS_GELU  epi(x) = GELU(x + bias[j]),  GELU(u) = u/2 (1 + erf(u / sqrt 2))
+ *
+ *   a         device, bf16 [M, K] row-major, 16-byte aligned, read only (may be NULL if K = 0).
+ *   b         device, bf16 [K, N] row-major, 16-byte aligned, read only (may be NULL if K = 0).
+ *   bias      device, bf16 [N], 16-byte aligned, read only; unused (may be NULL) with
+ *             FA_GEMM_PLAIN.
+ *   c         device, bf16 [M, N] row-major, 16-byte aligned, written; must not overlap a, b
+ *             or bias (not checked).
+ *   M, N, K   >= 0 and <= 2^31 - 256; N and K multiples of 8 (rows of whole 16-byte units).
+ *             M = 0 or N = 0 is a no-op returning FA_OK; K = 0 gives C = epi(0).
+ *   epilogue  a fa_gemm_epilogue value (FA_ERR_ARG otherwise).
+ *   dev_status  optional caller-owned device int, never cleared: receives FA_ERR_TIMEOUT if a
+ *             device-side pipeline wait ran out of time (about two seconds; C is then
+ *             undefined).  NULL to ignore.
+ *   stream    cudaStream_t or NULL.
+ * Checks, in order: epilogue (FA_ERR_ARG), negative sizes (FA_ERR_SHAPE), empty (FA_OK),
+ * pointers (FA_ERR_NULL), size limits and multiples of 8 (FA_ERR_SHAPE), alignment
+ * (FA_ERR_ALIGN), device (FA_ERR_ARCH / FA_ERR_CUDA).  Arithmetic: bf16 products with fp32
+ * accumulation in tensor memory, the epilogue in fp32, C rounded to bf16 (nearest-even).
+ * One launch, asynchronous on `stream`; nothing is allocated.
+ */
+int fa_gemm(const void* a, const void* b, const void* bias, void* c, int64_t M, int64_t N,
+            int64_t K, int epilogue, int* dev_status, void* stream);
+
+/* Number of kernel launches one fa_gemm call makes (0 or 1). */
+int fa_gemm_launches(int64_t M, int64_t N, int64_t K);
+
+/*
+ * fa_vector_add - z[i] = x[i] + y[i] over fp32 (the tutorial's vector-add
+ * kernel, a memory-bandwidth probe).
+ *
+ *   x, y  device, fp32 [n], read only, 4-byte aligned.
+ *   z     device, fp32 [n], written, 4-byte aligned; may be x or y itself (in place) but may
+ *         not overlap them otherwise.
+ *   n     0 .. 2^40 (0 is a no-op returning FA_OK; negative or larger: FA_ERR_SHAPE).
+ * IEEE fp32 addition, round-to-nearest-even, so the result is exact to the bit.  When all
+ * three pointers are 16-byte aligned the kernel moves 16-byte vectors, else single floats.
+ * Checks: size, pointers (FA_ERR_NULL), alignment (FA_ERR_ALIGN), device.  One launch,
+ * asynchronous on `stream`; nothing is allocated.
+ */
+int fa_vector_add(const float* x, const float* y, float* z, int64_t n, void* stream);
+
+/* Number of kernel launches one fa_vector_add call makes (0 or 1). */
+int fa_vector_add_launches(int64_t n);
 
 /* Number of kernel launches one fa_fwd call makes for these sizes (0 or 1). */
 int fa_fwd_launches(int64_t B, int64_t H, int64_t N, int64_t d);

@@ -107,6 +107,40 @@ def test_row_softmax_argument_checks():
     assert LIB.fa_row_softmax_launches(4, 8) == 1 and LIB.fa_row_softmax_launches(0, 8) == 0
 
 
+def test_gemm_argument_checks():
+    f = LIB.fa_gemm
+    P, B_, G = fa.FA_GEMM_PLAIN, fa.FA_GEMM_BIAS, fa.FA_GEMM_BIAS_GELU
+    assert f(16, 32, 48, 64, 8, 8, 8, 3, None, None) == fa.FA_ERR_ARG
+    assert f(16, 32, 48, 64, 8, 8, 8, -1, None, None) == fa.FA_ERR_ARG
+    assert f(16, 32, 48, 64, -1, 8, 8, G, None, None) == fa.FA_ERR_SHAPE
+    assert f(16, 32, 48, 64, 8, 8, -8, G, None, None) == fa.FA_ERR_SHAPE
+    assert f(None, None, None, None, 0, 8, 8, G, None, None) == fa.FA_OK      # empty: no-op
+    assert f(None, None, None, None, 8, 0, 8, G, None, None) == fa.FA_OK
+    assert f(16, 32, 48, None, 8, 8, 8, G, None, None) == fa.FA_ERR_NULL
+    assert f(None, 32, 48, 64, 8, 8, 8, G, None, None) == fa.FA_ERR_NULL
+    assert f(16, 32, None, 64, 8, 8, 8, B_, None, None) == fa.FA_ERR_NULL    # bias needed
+    assert f(16, 32, 48, 64, 8, 12, 8, G, None, None) == fa.FA_ERR_SHAPE     # N % 8
+    assert f(16, 32, 48, 64, 8, 8, 12, G, None, None) == fa.FA_ERR_SHAPE     # K % 8
+    assert f(16, 32, 48, 64, 2 ** 31, 8, 8, G, None, None) == fa.FA_ERR_SHAPE
+    assert f(18, 32, 48, 64, 8, 8, 8, G, None, None) == fa.FA_ERR_ALIGN
+    assert f(16, 32, 50, 64, 8, 8, 8, G, None, None) == fa.FA_ERR_ALIGN
+    assert f(16, 32, 48, 66, 8, 8, 8, G, None, None) == fa.FA_ERR_ALIGN
+    # K = 0 needs neither A nor B; the plain epilogue needs no bias (checks then pass to the device)
+    assert f(None, None, 48, 66, 8, 8, 0, G, None, None) == fa.FA_ERR_ALIGN
+    assert f(16, 32, None, 66, 8, 8, 8, P, None, None) == fa.FA_ERR_ALIGN
+    assert LIB.fa_gemm_launches(8, 8, 8) == 1 and LIB.fa_gemm_launches(0, 8, 8) == 0
+
+
+def test_vector_add_argument_checks():
+    f = LIB.fa_vector_add
+    assert f(16, 32, 48, -1, None) == fa.FA_ERR_SHAPE
+    assert f(None, None, None, 0, None) == fa.FA_OK
+    assert f(None, 32, 48, 4, None) == fa.FA_ERR_NULL
+    assert f(16, 32, 48, 2 ** 41, None) == fa.FA_ERR_SHAPE
+    assert f(18, 32, 48, 4, None) == fa.FA_ERR_ALIGN
+    assert LIB.fa_vector_add_launches(5) == 1 and LIB.fa_vector_add_launches(0) == 0
+
+
 def test_launch_count():
     assert fa.launches_per_call(1, 1, 128, 64) == 1
     assert fa.launches_per_call(0, 1, 128, 64) == 0
