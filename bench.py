@@ -89,6 +89,20 @@ def measured_traffic(workload):
         return None, None
 
 
+def profile_traffic(profile, source):
+    """DRAM bytes per launch from a committed ncu summary under profiles/, or
+    None when the kernel source changed since the capture."""
+    try:
+        text = open(os.path.join(ROOT, "profiles", profile)).read()
+        want = re.search(r"kernel_source_sha256_16: (\w+)", text).group(1)
+        have = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
+        if want != have:
+            return None
+        return float(re.search(r"traffic_bytes_per_launch: ([0-9.e+]+)", text).group(1))
+    except (OSError, AttributeError, ValueError):
+        return None
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -448,7 +462,9 @@ def bench_row_softmax(args):
             "data": "synthetic", "config": {"workload": f"row_softmax_r{rows}_c{cols}", "rows": rows,
                                             "cols": cols, "l2": "512 MiB moved per launch, above L2"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm"], "traffic": None,
+                         "frac": gbs / peaks["hbm"],
+                         "traffic": profile_traffic("row_softmax_fast_r32768_c4096_ncu.md",
+                                                    "attention_forward_17_b200/csrc/row_softmax.cu"),
                          "algorithmic_bytes_per_launch": nbytes},
             "cpu_baseline": {"value": sample * cols * 4 / dt / 1e9, "unit": "GB/s",
                              "cores": oracle.default_threads(), "kind": "oracle",
@@ -520,7 +536,9 @@ def bench_gemm(args):
             "config": {"workload": f"gemm_bias_gelu_m{M}_n{N}_k{K}", "M": M, "N": N, "K": K,
                        "l2": "A, B, C = 384 MiB, above L2"},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16"],
-                         "unit": "TFLOP/s", "frac": tf / peaks["bf16"], "traffic": None,
+                         "unit": "TFLOP/s", "frac": tf / peaks["bf16"],
+                         "traffic": profile_traffic("gemm_kernel_m8192_n8192_k8192_ncu.md",
+                                                    "attention_forward_17_b200/csrc/gemm_bias_gelu.cu"),
                          "algorithmic_flops_per_launch": flop,
                          "peak_source": peaks["source"] + " bf16 burst (cuBLAS 8192^3)"},
             "context": {"cublas_plain_tflops": flop / (ms_plain / 1e3) / 1e12,
@@ -563,7 +581,9 @@ def bench_vector_add(args):
             "data": "synthetic", "config": {"workload": f"vector_add_n{n}", "n": n,
                                             "l2": "3 GiB moved per launch, above L2"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm"], "traffic": None,
+                         "frac": gbs / peaks["hbm"],
+                         "traffic": profile_traffic("vector_add_v4_n268435456_ncu.md",
+                                                    "attention_forward_17_b200/csrc/vector_add.cu"),
                          "algorithmic_bytes_per_launch": nbytes},
             "cpu_baseline": {"value": m * 12.0 / dt / 1e9, "unit": "GB/s",
                              "cores": oracle.default_threads(), "kind": "oracle",
