@@ -62,6 +62,15 @@ def _load():
     lib.fa_row_softmax.restype = ctypes.c_int
     lib.fa_row_softmax_launches.argtypes = [_i64, _i64]
     lib.fa_row_softmax_launches.restype = ctypes.c_int
+    lib.fa_fwd_schedule.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.c_int,
+                                    ctypes.c_float, ctypes.c_int, ctypes.c_int, _vp, _vp]
+    lib.fa_fwd_schedule.restype = ctypes.c_int
+    lib.fa_schedule_count.argtypes = []
+    lib.fa_schedule_count.restype = ctypes.c_int
+    lib.fa_schedule_info.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp]
+    lib.fa_schedule_info.restype = ctypes.c_int
+    lib.fa_fwd_pick_schedule.argtypes = [_i64, _i64, ctypes.c_int, _vp, _vp]
+    lib.fa_fwd_pick_schedule.restype = ctypes.c_int
     lib.fa_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, ctypes.c_int, _vp, _vp]
     lib.fa_gemm.restype = ctypes.c_int
     lib.fa_gemm_launches.argtypes = [_i64, _i64, _i64]
@@ -119,14 +128,38 @@ def _check_qkv(q, k, v):
         raise ValueError("q, k, v must be on the same CUDA device")
 
 
+def schedules() -> list[dict]:
+    """Every compiled schedule of the attention kernel: id, d, emu_every, kv_slots, smem_bytes."""
+    out = []
+    for i in range(lib.fa_schedule_count()):
+        vals = [ctypes.c_int() for _ in range(4)]
+        rc = lib.fa_schedule_info(i, *[ctypes.byref(x) for x in vals])
+        if rc != FA_OK:
+            raise FaError(rc, "fa_schedule_info")
+        out.append(dict(id=i, d=vals[0].value, emu_every=vals[1].value, kv_slots=vals[2].value,
+                        smem_bytes=vals[3].value))
+    return out
+
+
+def pick_schedule(N: int, d: int, causal: bool) -> tuple[int, int]:
+    """(schedule id, causal group) that fa_fwd uses for this problem."""
+    sid, grp = ctypes.c_int(), ctypes.c_int()
+    rc = lib.fa_fwd_pick_schedule(N, d, int(bool(causal)), ctypes.byref(sid), ctypes.byref(grp))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_pick_schedule")
+    return sid.value, grp.value
+
+
 def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
-           stream=None, status=None):
+           stream=None, status=None, schedule: int | None = None, causal_group: int | None = None):
     """O, LSE = attention forward of bf16 [B, H, N, d] CUDA tensors.
 
     ``out`` (bf16 [B,H,N,d]) and ``lse`` (fp32 [B,H,N]) are allocated when not
     given.  Runs on ``stream`` (a torch.cuda.Stream) or the current stream.
     ``status`` may be an int32 CUDA tensor with one element; it then receives
-    FA_ERR_TIMEOUT should a device-side wait run out of time.
+    FA_ERR_TIMEOUT should a device-side wait run out of time.  ``schedule``
+    (an id from ``schedules()``) and ``causal_group`` override the table's
+    choice.
     """
     import torch
     _check_qkv(q, k, v)
@@ -143,7 +176,13 @@ def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, 
         raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
     s = (stream if stream is not None else torch.cuda.current_stream(q.device)).cuda_stream
     with torch.cuda.device(q.device):
-        if status is None:
+        if schedule is not None or causal_group is not None:
+            rc = lib.fa_fwd_schedule(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                     lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                     -1 if schedule is None else int(schedule),
+                                     0 if causal_group is None else int(causal_group),
+                                     status.data_ptr() if status is not None else None, s)
+        elif status is None:
             rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                             lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale), s)
         else:

@@ -28,7 +28,8 @@ def library_path() -> str:
 
 def _sources():
     return [os.path.join(CSRC, f) for f in
-            ("fa_fwd.cu", "row_softmax.cu", "gemm_bias_gelu.cu", "vector_add.cu")]
+            ("fa_fwd.cu", "fa_fwd_sched_d128.cu", "fa_fwd_sched_d64.cu", "row_softmax.cu",
+             "gemm_bias_gelu.cu", "vector_add.cu")]
 
 
 def _deps():
@@ -43,13 +44,33 @@ def build(force: bool = False, verbose: bool = False) -> str:
             and all(os.path.getmtime(out) >= os.path.getmtime(p) for p in _deps())):
         return out
     nvcc = os.environ.get("NVCC", "nvcc")
+    objdir = os.path.join(HERE, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    inc = ["-I", os.path.join(ROOT, "include")]
+    flags = [f for f in NVCC_FLAGS if f != "-shared"]
+
+    def compile_one(src):
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        cmd = [nvcc, *flags, *inc, "-c", src, "-o", obj]
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        return obj, " ".join(cmd) + "\n" + res.stdout + res.stderr, res.returncode
+
+    # the translation units compile independently; run them side by side
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as pool:
+        results = list(pool.map(compile_one, _sources()))
+    log = "".join(r[1] for r in results)
+    failed = any(r[2] != 0 for r in results)
     tmp = out + ".tmp"
-    cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), *_sources(), "-o", tmp]
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    log = res.stdout + res.stderr
+    if not failed:
+        cmd = [nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
+               *[r[0] for r in results], "-o", tmp]
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        log += " ".join(cmd) + "\n" + res.stdout + res.stderr
+        failed = res.returncode != 0
     with open(os.path.join(HERE, "build.log"), "w") as f:
-        f.write(" ".join(cmd) + "\n" + log)
-    if res.returncode != 0:
+        f.write(log)
+    if failed:
         sys.stderr.write(log)
         raise RuntimeError("nvcc failed building libfa_b200.so")
     if verbose:

@@ -11,7 +11,30 @@
 
 #include "../../include/fa.h"
 #include "fa_fwd_kernel.cuh"
+#include "fa_schedule_table.h"
+#include "fa_schedules.h"
 #include "host_common.h"
+
+namespace fa {
+// Exercises the bounded wait on an mbarrier that nothing ever arrives at: the
+// wait must give up after `limit_ns` and leave FA_ERR_TIMEOUT in *status.
+// With `arrive` set, one thread completes the phase first and the wait must
+// return at once with *status untouched.  One CTA of 32 threads.
+__global__ void fa_wait_selftest_kernel(int* status, uint64_t limit_ns, int arrive) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0u;
+        fence_barrier_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0 && arrive) mbar_arrive(smem_u32(&bar));
+    __syncwarp();
+    if (!mbar_try_wait(smem_u32(&bar), 0))
+        wait_slow(smem_u32(&bar), 0, &abort_flag, status, limit_ns, limit_ns);
+}
+}  // namespace fa
 
 namespace {
 
@@ -25,20 +48,22 @@ DeviceState g_devices[kMaxDevices];
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
-// Opts the instantiation into its dynamic shared memory and checks that it was
-// compiled with enough registers for the in-kernel warpgroup rebalance (a
-// setmaxnreg.inc asking for more than the launch allocated would never
-// return).
-template <int D, bool CAUSAL>
-int set_smem_attr() {
-    if (cudaFuncSetAttribute(fa::fa_fwd_kernel<D, CAUSAL>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fa::TileCfg<D>::kSmemBytes) != cudaSuccess)
-        return FA_ERR_CUDA;
-    cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, fa::fa_fwd_kernel<D, CAUSAL>) != cudaSuccess) return FA_ERR_CUDA;
-    if (attr.numRegs * fa::kThreads < fa::kRegSplitTotal) return FA_ERR_CUDA;
-    return FA_OK;
+// Every compiled schedule, head dimension 128 first, then 64.  Ids are
+// positions in this list.
+struct ScheduleList {
+    const fa::Schedule* items[64];
+    int count = 0;
+    ScheduleList() {
+        int n = 0;
+        const fa::Schedule* a = fa::schedules_d128(&n);
+        for (int i = 0; i < n && count < 64; ++i) items[count++] = &a[i];
+        const fa::Schedule* b = fa::schedules_d64(&n);
+        for (int i = 0; i < n && count < 64; ++i) items[count++] = &b[i];
+    }
+};
+const ScheduleList& schedules() {
+    static const ScheduleList list;
+    return list;
 }
 
 // One-time per-device set-up: architecture check and the shared-memory opt-in
@@ -49,11 +74,37 @@ int device_setup(int dev) {
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
         return FA_ERR_CUDA;
     if (major != 10 || minor != 0) return FA_ERR_ARCH;
-    int rc;
-    if ((rc = set_smem_attr<64, false>()) != FA_OK || (rc = set_smem_attr<64, true>()) != FA_OK ||
-        (rc = set_smem_attr<128, false>()) != FA_OK || (rc = set_smem_attr<128, true>()) != FA_OK)
-        return rc;
+    const ScheduleList& list = schedules();
+    for (int i = 0; i < list.count; ++i) {
+        const int rc = list.items[i]->setup();
+        if (rc != FA_OK) return rc;
+    }
     return FA_OK;
+}
+
+// The schedule id fa_fwd uses for (N, d, causal), and the causal launch group.
+void pick_schedule(int64_t N, int64_t d, int causal, int* id, int* group) {
+    const ScheduleList& list = schedules();
+    int emu = -1, slots = -1, grp = 1;
+    for (const auto& e : fa::kScheduleTable)
+        if (e.d == d && e.causal == (causal ? 1 : 0) && N <= e.n_max) {
+            emu = e.emu;
+            slots = e.slots;
+            grp = e.group;
+            break;
+        }
+    int first = -1, match = -1;
+    for (int i = 0; i < list.count; ++i) {
+        const fa::Schedule* s = list.items[i];
+        if (s->d != d) continue;
+        if (first < 0) first = i;
+        if (s->emu == emu && s->slots == slots) {
+            match = i;
+            break;
+        }
+    }
+    *id = match >= 0 ? match : first;
+    *group = grp > 0 ? grp : 1;
 }
 
 int current_device_ready() {
@@ -105,19 +156,20 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
     return 0;
 }
 
-template <int D, bool CAUSAL>
-cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const fa::FwdParams& p, int64_t grid, cudaStream_t stream) {
-    fa::fa_fwd_kernel<D, CAUSAL><<<static_cast<unsigned>(grid), fa::kThreads,
-                                   fa::TileCfg<D>::kSmemBytes, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError();
-}
-
+// schedule_id < 0 and group < 1 take the table's choice.
 int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
-            int64_t N, int64_t d, int causal, float scale, int* dev_status, void* stream) {
+            int64_t N, int64_t d, int causal, float scale, int schedule_id, int group,
+            int* dev_status, void* stream) {
     int rc = check_args(q, k, v, o, lse, B, H, N, d, scale);
     if (rc == 1) return FA_OK;
     if (rc != 0) return rc;
+    const ScheduleList& list = schedules();
+    if (schedule_id >= list.count || (schedule_id >= 0 && list.items[schedule_id]->d != d))
+        return FA_ERR_ARG;
+    int table_id = 0, table_group = 1;
+    pick_schedule(N, d, causal, &table_id, &table_group);
+    if (schedule_id < 0) schedule_id = table_id;
+    if (group < 1) group = table_group;
     if ((rc = current_device_ready()) != FA_OK) return rc;
     if ((rc = encoder_ready()) != FA_OK) return rc;
     const int64_t BH = B * H;
@@ -132,16 +184,13 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
     p.N = static_cast<int>(N);
     p.BH = static_cast<int>(BH);
     p.n_qtile = static_cast<int>((N + fa::kBlockM - 1) / fa::kBlockM);
+    p.group = static_cast<int>(group < BH ? group : BH);
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     const int64_t grid = BH * p.n_qtile;
     if (grid > 0x7fffffffLL) return FA_ERR_SHAPE;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e;
-    if (d == 64)
-        e = causal ? launch<64, true>(tq, tk, tv, p, grid, s) : launch<64, false>(tq, tk, tv, p, grid, s);
-    else
-        e = causal ? launch<128, true>(tq, tk, tv, p, grid, s)
-                   : launch<128, false>(tq, tk, tv, p, grid, s);
+    const fa::Schedule* sch = list.items[schedule_id];
+    const cudaError_t e = sch->launch[causal ? 1 : 0](tq, tk, tv, p, static_cast<unsigned>(grid),
+                                                       static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -151,13 +200,45 @@ extern "C" {
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
            int64_t N, int64_t d, int causal, float scale, void* stream) {
-    return run_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, nullptr, stream);
+    return run_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, -1, 0, nullptr, stream);
 }
 
 int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
                   int64_t H, int64_t N, int64_t d, int causal, float scale, int* dev_status,
                   void* stream) {
-    return run_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, dev_status, stream);
+    return run_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, -1, 0, dev_status, stream);
+}
+
+int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                    int64_t H, int64_t N, int64_t d, int causal, float scale, int schedule_id,
+                    int causal_group, int* dev_status, void* stream) {
+    if (schedule_id < -1 || causal_group < 0) {
+        const int rc = check_args(q, k, v, o, lse, B, H, N, d, scale);
+        return rc == 0 ? FA_ERR_ARG : (rc == 1 ? FA_OK : rc);
+    }
+    return run_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, schedule_id, causal_group,
+                   dev_status, stream);
+}
+
+int fa_schedule_count(void) { return schedules().count; }
+
+int fa_schedule_info(int id, int* d, int* emu_every, int* kv_slots, int* smem_bytes) {
+    const ScheduleList& list = schedules();
+    if (id < 0 || id >= list.count) return FA_ERR_ARG;
+    const fa::Schedule* s = list.items[id];
+    if (d) *d = s->d;
+    if (emu_every) *emu_every = s->emu;
+    if (kv_slots) *kv_slots = s->slots;
+    if (smem_bytes) *smem_bytes = s->smem_bytes;
+    return FA_OK;
+}
+
+int fa_fwd_pick_schedule(int64_t N, int64_t d, int causal, int* schedule_id, int* causal_group) {
+    if (!schedule_id || !causal_group) return FA_ERR_NULL;
+    if (N < 0) return FA_ERR_SHAPE;
+    if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+    pick_schedule(N, d, causal, schedule_id, causal_group);
+    return FA_OK;
 }
 
 int fa_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, float* lse_h,
@@ -174,7 +255,7 @@ int fa_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, fl
         cudaMemcpyAsync(k_d, k_h, tensor_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(v_d, v_h, tensor_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return FA_ERR_CUDA;
-    rc = run_fwd(q_d, k_d, v_d, o_d, lse_d, B, H, N, d, causal, scale, nullptr, stream);
+    rc = run_fwd(q_d, k_d, v_d, o_d, lse_d, B, H, N, d, causal, scale, -1, 0, nullptr, stream);
     if (rc != FA_OK) return rc;
     if (cudaMemcpyAsync(o_h, o_d, tensor_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaMemcpyAsync(lse_h, lse_d, lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)

@@ -68,12 +68,6 @@ constexpr uint64_t kWaitLimitAbortNs = 1000000ull;    // 1 ms once the CTA has a
 constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kRegsOther = 88;
 constexpr int kRegSplitTotal = 2 * 128 * kRegsSoftmax + 128 * kRegsOther;  // 64512 = 384 x 168
-// Every kEmuEvery-th pair of exponentials is evaluated on the FMA pipe by
-// polynomial instead of on the special-function unit (0 = never).
-#ifndef FA_EMU_EVERY
-#define FA_EMU_EVERY 4
-#endif
-constexpr int kEmuEvery = FA_EMU_EVERY;
 // Sum the bf16-rounded weights with mixed-precision adds that read the 16-bit
 // halves directly (1) or by widening the halves to fp32 first (0).
 #ifndef FA_LHAT_MIXED_ADD
@@ -85,13 +79,26 @@ constexpr int kEmuEvery = FA_EMU_EVERY;
 #define FA_SOFTMAX_PHASED 1
 #endif
 
-template <int D>
+// Schedule knobs (template parameters of the kernel, chosen per problem by
+// the host from a table the schedule search writes):
+//   EMU    every EMU-th pair of exponentials is evaluated on the FMA pipe by
+//          polynomial instead of on the special-function unit (0 = never);
+//   SLOTS  depth of the K/V shared-memory ring.
+template <int D, int SLOTS>
 struct TileCfg {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    // A parity wait on a ring slot is only sound if the slot's previous load
+    // has already landed when the wait starts (else the wait can mistake that
+    // older phase for the one it wants).  The score issuer waits K_m after
+    // PV(m-3) completed and the output issuer waits V_t after P_t, which
+    // cover every earlier load that can share the slot once the ring holds
+    // at least four tiles: V_t (sequence position 2t+3) then shares a slot
+    // with V_{t'<t} or K_{m<=t} only.  With three slots V_t would share K_{t+1}'s.
+    static_assert(SLOTS >= 4, "K/V ring depth");
     static constexpr int kTileBytes = kBlockN * D * 2;      // one K or V tile (bf16)
     static constexpr int kBoxes = D / 64;                   // 64-column (128-byte) TMA boxes
     static constexpr int kBoxBytes = 128 * 128;             // 128 rows x 128 bytes
-    static constexpr int kSlots = (D == 128) ? 5 : 8;       // K/V ring depth
+    static constexpr int kSlots = SLOTS;                    // K/V ring depth
     static constexpr int kQOff = 0;
     static constexpr int kSlotOff = kTileBytes;             // after the Q tile
     static constexpr int kBarOff = kSlotOff + kSlots * kTileBytes;
@@ -123,6 +130,7 @@ struct FwdParams {
     int N;
     int BH;
     int n_qtile;             // ceil(N / 128)
+    int group;               // causal launch order: heads per group (>= 1)
     float scale_log2;        // scale * log2(e)
 };
 
@@ -163,25 +171,6 @@ __device__ __forceinline__ void wait_bar(uint32_t bar, uint32_t parity, volatile
         wait_slow(bar, parity, abort, status, kWaitLimitNs, kWaitLimitAbortNs);
 }
 
-// Exercises the bounded wait on an mbarrier that nothing ever arrives at: the
-// wait must give up after `limit_ns` and leave FA_ERR_TIMEOUT in *status.
-// With `arrive` set, one thread completes the phase first and the wait must
-// return at once with *status untouched.  One CTA of 32 threads.
-__global__ void fa_wait_selftest_kernel(int* status, uint64_t limit_ns, int arrive) {
-    __shared__ __align__(8) uint64_t bar;
-    __shared__ uint32_t abort_flag;
-    if (threadIdx.x == 0) {
-        mbar_init(smem_u32(&bar), 1);
-        abort_flag = 0u;
-        fence_barrier_init();
-    }
-    __syncwarp();
-    if (threadIdx.x == 0 && arrive) mbar_arrive(smem_u32(&bar));
-    __syncwarp();
-    if (!mbar_try_wait(smem_u32(&bar), 0))
-        wait_slow(smem_u32(&bar), 0, &abort_flag, status, limit_ns, limit_ns);
-}
-
 // ---------------------------------------------------------------- exp2 on the FMA pipe
 // 2^x for two values without the special-function unit (Cody-Waite style
 // split x = j + f):
@@ -215,11 +204,11 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, int EMU, int SLOTS>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using C = TileCfg<D>;
+    using C = TileCfg<D, SLOTS>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -231,12 +220,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: CTAs of one (b, h) slice are adjacent in launch order so the
-    // slice's K/V stay in L2; under the causal mask the longest query tiles of
-    // a slice launch first.
-    const int bh = blockIdx.x / p.n_qtile;
-    const int qi = blockIdx.x % p.n_qtile;
-    const int qt = CAUSAL ? (p.n_qtile - 1 - qi) : qi;
+    // Work item.  Without the mask, the CTAs of one (b, h) slice are adjacent
+    // in launch order so the slice's K/V stay in L2.  Under the causal mask the
+    // slices are taken `group` at a time and, inside a group, query tiles are
+    // launched longest first (all the group's last tiles, then the tiles before
+    // them, ...), which keeps the group's K/V in L2 while the short tiles fill
+    // the end of the grid.
+    int bh, qt;
+    if constexpr (CAUSAL) {
+        const int span = p.group * p.n_qtile;
+        const int g0 = (blockIdx.x / span) * p.group;
+        const int heads = min(p.group, p.BH - g0);
+        const int r = blockIdx.x % span;
+        bh = g0 + r % heads;
+        qt = p.n_qtile - 1 - r / heads;
+    } else {
+        bh = blockIdx.x / p.n_qtile;
+        qt = blockIdx.x % p.n_qtile;
+    }
     const int q0 = qt * kBlockM;
     const int n_kv_all = (p.N + kBlockN - 1) / kBlockN;
     const int n_kv = CAUSAL ? min(n_kv_all, qt + 1) : n_kv_all;
@@ -421,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < 32; ++i) {
                     const int o = 4 * (i >> 1) + 2 * (i & 1);
                     float p0, p1;
-                    if (kEmuEvery > 0 && (i % kEmuEvery) == kEmuEvery - 1) {
+                    if (EMU > 0 && (i % (EMU > 0 ? EMU : 1)) == EMU - 1) {
                         exp2_poly2(__uint_as_float(s[o]), __uint_as_float(s[o + 1]), p0, p1);
                     } else {
                         p0 = ex2_approx(__uint_as_float(s[o]));
@@ -458,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float x0, x1;
                 f2_split(x2, x0, x1);
                 float p0, p1;
-                if (kEmuEvery > 0 && (i % kEmuEvery) == kEmuEvery - 1) {
+                if (EMU > 0 && (i % (EMU > 0 ? EMU : 1)) == EMU - 1) {
                     exp2_poly2(x0, x1, p0, p1);
                 } else {
                     p0 = ex2_approx(x0);
@@ -646,9 +647,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int t = 0; t < n_kv; ++t) {
                     const int b = t % kSBufs;
                     const int iv = load_index_v(t, n_kv);
-                    wait_kv(iv);
+                    // P_t first: it implies that every K_m (m <= t) has landed,
+                    // which the parity wait on V_t's slot relies on (see
+                    // TileCfg).
                     wait_bar(bar_p_full + 8 * b, (t / kSBufs) & 1, abort, p.status);
-                    tc_fence_after();
+                    wait_kv(iv);
                     const uint64_t b0 = desc_v + (slot_addr(iv) >> 4);
                     const uint32_t a_tmem = tmem + C::col_s(b) + C::kColP;
 #pragma unroll

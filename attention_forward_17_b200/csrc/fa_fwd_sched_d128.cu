@@ -1,0 +1,21 @@
+// Compiled schedules of the attention kernel for head dimension 128: the
+// exponential split (EMU) times the K/V ring depth (SLOTS), every combination
+// that fits 227 KiB of shared memory (a slot is one 32 KiB K or V tile, the Q
+// tile takes another 32 KiB, so at most five slots; at least four keep the
+// ring's parity waits sound).  First entry = default.
+#include "fa_schedules.h"
+
+namespace fa {
+namespace {
+const Schedule kD128[] = {
+    make_schedule<128, 4, 5>(), make_schedule<128, 0, 5>(), make_schedule<128, 2, 5>(),
+    make_schedule<128, 4, 4>(), make_schedule<128, 0, 4>(), make_schedule<128, 2, 4>(),
+};
+}  // namespace
+
+const Schedule* schedules_d128(int* count) {
+    *count = static_cast<int>(sizeof(kD128) / sizeof(kD128[0]));
+    return kD128;
+}
+
+}  // namespace fa

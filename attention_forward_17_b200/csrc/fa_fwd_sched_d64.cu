@@ -1,0 +1,19 @@
+// Compiled schedules of the attention kernel for head dimension 64: the
+// exponential split (EMU) times the K/V ring depth (SLOTS, 16 KiB a slot).
+// First entry = default.
+#include "fa_schedules.h"
+
+namespace fa {
+namespace {
+const Schedule kD64[] = {
+    make_schedule<64, 4, 8>(), make_schedule<64, 0, 8>(), make_schedule<64, 2, 8>(),
+    make_schedule<64, 4, 4>(), make_schedule<64, 0, 4>(), make_schedule<64, 2, 4>(),
+};
+}  // namespace
+
+const Schedule* schedules_d64(int* count) {
+    *count = static_cast<int>(sizeof(kD64) / sizeof(kD64[0]));
+    return kD64;
+}
+
+}  // namespace fa

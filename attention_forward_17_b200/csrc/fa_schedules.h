@@ -1,0 +1,75 @@
+// Registry of the compiled schedules of the attention kernel.  A schedule is
+// one instantiation of fa_fwd_kernel<D, CAUSAL, EMU, SLOTS> for both masking
+// modes; the host picks one per problem from the table the schedule search
+// writes (fa_schedule_table.h) or as the caller asks (fa_fwd_schedule).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa_fwd_kernel.cuh"
+
+namespace fa {
+
+using FwdLaunchFn = cudaError_t (*)(const CUtensorMap& tq, const CUtensorMap& tk,
+                                    const CUtensorMap& tv, const FwdParams& p, unsigned grid,
+                                    cudaStream_t stream);
+
+struct Schedule {
+    int d;             // head dimension
+    int emu;           // every emu-th exponential pair on the FMA pipe (0 = none)
+    int slots;         // K/V ring depth
+    int smem_bytes;    // dynamic shared memory per CTA
+    FwdLaunchFn launch[2];   // [causal]
+    int (*setup)();          // shared-memory opt-in and register check, both modes
+};
+
+// Defined in fa_fwd_sched_d128.cu and fa_fwd_sched_d64.cu; the first entry of
+// each list is that head dimension's default.
+const Schedule* schedules_d128(int* count);
+const Schedule* schedules_d64(int* count);
+
+// Shared by both definition files.
+template <int D, bool CAUSAL, int EMU, int SLOTS>
+cudaError_t launch_schedule(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FwdParams& p, unsigned grid, cudaStream_t stream) {
+    fa_fwd_kernel<D, CAUSAL, EMU, SLOTS>
+        <<<grid, kThreads, TileCfg<D, SLOTS>::kSmemBytes, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+// Opts the instantiation into its dynamic shared memory and checks that it
+// was compiled with enough registers for the in-kernel warpgroup rebalance (a
+// setmaxnreg.inc asking for more than the launch allocated would never
+// return).  Returns 0 (FA_OK), -6 (FA_ERR_CUDA).
+template <int D, bool CAUSAL, int EMU, int SLOTS>
+int setup_one() {
+    auto* k = fa_fwd_kernel<D, CAUSAL, EMU, SLOTS>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             TileCfg<D, SLOTS>::kSmemBytes) != cudaSuccess)
+        return -6;
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, k) != cudaSuccess) return -6;
+    if (attr.numRegs * kThreads < kRegSplitTotal) return -6;
+    return 0;
+}
+
+template <int D, int EMU, int SLOTS>
+int setup_both() {
+    const int rc = setup_one<D, false, EMU, SLOTS>();
+    return rc ? rc : setup_one<D, true, EMU, SLOTS>();
+}
+
+template <int D, int EMU, int SLOTS>
+constexpr Schedule make_schedule() {
+    static_assert(TileCfg<D, SLOTS>::kSmemBytes <= 232448, "shared memory per CTA (227 KiB)");
+    static_assert(TileCfg<D, SLOTS>::kTmemCols <= 512, "tensor memory columns");
+    return Schedule{D,
+                    EMU,
+                    SLOTS,
+                    TileCfg<D, SLOTS>::kSmemBytes,
+                    {&launch_schedule<D, false, EMU, SLOTS>, &launch_schedule<D, true, EMU, SLOTS>},
+                    &setup_both<D, EMU, SLOTS>};
+}
+
+}  // namespace fa

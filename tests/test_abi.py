@@ -141,6 +141,45 @@ def test_vector_add_argument_checks():
     assert LIB.fa_vector_add_launches(5) == 1 and LIB.fa_vector_add_launches(0) == 0
 
 
+def test_schedule_registry():
+    n = LIB.fa_schedule_count()
+    assert n >= 2
+    import ctypes
+    vals = [ctypes.c_int() for _ in range(4)]
+    seen = set()
+    for i in range(n):
+        assert LIB.fa_schedule_info(i, *[ctypes.byref(x) for x in vals]) == fa.FA_OK
+        d, emu, slots, smem = (x.value for x in vals)
+        assert d in (64, 128) and emu in (0, 2, 4) and slots >= 2 and 0 < smem <= 232448
+        assert (d, emu, slots) not in seen
+        seen.add((d, emu, slots))
+    assert LIB.fa_schedule_info(n, None, None, None, None) == fa.FA_ERR_ARG
+    assert LIB.fa_schedule_info(-1, None, None, None, None) == fa.FA_ERR_ARG
+    # the first schedule of each head dimension is the default
+    assert fa.schedules()[0]["d"] == 128
+
+
+def test_schedule_argument_checks():
+    f = LIB.fa_fwd_schedule
+    args = (16, 32, 48, 64, 80, 1, 1, 128)
+    n = LIB.fa_schedule_count()
+    d64 = [s["id"] for s in fa.schedules() if s["d"] == 64][0]
+    assert f(*args, 128, 0, 0.125, n, 1, None, None) == fa.FA_ERR_ARG     # unknown id
+    assert f(*args, 128, 0, 0.125, d64, 1, None, None) == fa.FA_ERR_ARG   # id for another d
+    assert f(*args, 128, 0, 0.125, -2, 1, None, None) == fa.FA_ERR_ARG
+    assert f(*args, 128, 1, 0.125, 0, -1, None, None) == fa.FA_ERR_ARG
+    # the attention arguments are checked first
+    assert f(*args[:5], -1, 1, 128, 128, 0, 0.125, n, 1, None, None) == fa.FA_ERR_SHAPE
+    assert f(*args[:5], 0, 1, 128, 128, 0, 0.125, n, 1, None, None) == fa.FA_OK
+    assert f(*args, 96, 0, 0.125, 0, 1, None, None) == fa.FA_ERR_HEADDIM
+    import ctypes
+    sid, grp = ctypes.c_int(), ctypes.c_int()
+    assert LIB.fa_fwd_pick_schedule(4096, 128, 1, ctypes.byref(sid), ctypes.byref(grp)) == fa.FA_OK
+    assert LIB.fa_fwd_pick_schedule(4096, 128, 1, None, ctypes.byref(grp)) == fa.FA_ERR_NULL
+    assert LIB.fa_fwd_pick_schedule(-1, 128, 1, ctypes.byref(sid), ctypes.byref(grp)) == fa.FA_ERR_SHAPE
+    assert LIB.fa_fwd_pick_schedule(64, 80, 1, ctypes.byref(sid), ctypes.byref(grp)) == fa.FA_ERR_HEADDIM
+
+
 def test_launch_count():
     assert fa.launches_per_call(1, 1, 128, 64) == 1
     assert fa.launches_per_call(0, 1, 128, 64) == 0

@@ -1,0 +1,70 @@
+"""Every compiled schedule of the attention kernel against the fp64 oracle
+(ragged N, both masking modes, wide score range), the causal launch groups
+(including a group size that does not divide B*H, so the last group is
+partial: a tile launched twice or never would show), and the table's choice
+for each problem class."""
+import numpy as np
+import pytest
+
+import oracle
+import parity_utils as pu
+
+pytestmark = pytest.mark.gpu
+
+
+def _schedules():
+    import attention_forward_17_b200 as fa
+    return fa.schedules()
+
+
+def run_sched(qt, kt, vt, causal, sid, group):
+    import torch
+    import attention_forward_17_b200 as fa
+    o, lse = fa.fa_fwd(qt, kt, vt, causal, schedule=sid, causal_group=group)
+    torch.cuda.synchronize()
+    return pu.o_f64(o), lse.double().cpu().numpy()
+
+
+@pytest.mark.parametrize("sid", range(15))
+def test_every_schedule_matches_oracle(cuda_device, sid):
+    sched = _schedules()
+    if sid >= len(sched):
+        pytest.skip("fewer schedules compiled")
+    d = sched[sid]["d"]
+    (q, k, v), (qt, kt, vt) = pu.inputs(1, 2, 1000, d, seed=sid, sigma_qk=3.0)
+    for causal in (False, True):
+        o_ref, lse_ref = oracle.attention_fwd(q, k, v, causal, pu.default_scale(d))
+        o, lse = run_sched(qt, kt, vt, causal, sid, 1)
+        pu.check(o, lse, o_ref, lse_ref, f"schedule {sched[sid]} causal={causal}")
+
+
+@pytest.mark.parametrize("group", [1, 2, 3, 5, 64])
+def test_causal_groups_cover_every_tile(cuda_device, group):
+    # B*H = 5 slices of 5 query tiles (N = 600, last tile ragged)
+    (q, k, v), (qt, kt, vt) = pu.inputs(1, 5, 600, 64, seed=group)
+    o_ref, lse_ref = oracle.attention_fwd(q, k, v, True, pu.default_scale(64))
+    o, lse = run_sched(qt, kt, vt, True, 9, group)
+    pu.check(o, lse, o_ref, lse_ref, f"group {group}")
+
+
+def test_table_choice_is_valid():
+    import attention_forward_17_b200 as fa
+    sched = fa.schedules()
+    for d in (64, 128):
+        for causal in (False, True):
+            for N in (1, 1024, 2048, 2049, 4096, 8193, 16384, 1 << 20):
+                sid, grp = fa.pick_schedule(N, d, causal)
+                assert 0 <= sid < len(sched) and sched[sid]["d"] == d and grp >= 1
+
+
+def test_default_path_uses_the_table_choice(cuda_device):
+    # fa_fwd (no schedule) and fa_fwd_schedule with the table's pick are the same launch
+    import torch
+    import attention_forward_17_b200 as fa
+    (_, _, _), (qt, kt, vt) = pu.inputs(2, 3, 700, 128, seed=4)
+    for causal in (False, True):
+        sid, grp = fa.pick_schedule(700, 128, causal)
+        o1, l1 = fa.fa_fwd(qt, kt, vt, causal)
+        o2, l2 = fa.fa_fwd(qt, kt, vt, causal, schedule=sid, causal_group=grp)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
