@@ -278,10 +278,12 @@ def run_reference(args, cfg):
     print(json.dumps(line), flush=True)
 
 
-def schedule_of(N, d, causal):
-    """The kernel schedule fa_fwd uses for this problem (from the search table)."""
+def schedule_of(N, d, causal, schedule=None, causal_group=None):
+    """The kernel schedule used for this problem: the search table's, unless pinned."""
     import attention_forward_17_b200 as fa
     sid, grp = fa.pick_schedule(N, d, causal)
+    sid = sid if schedule is None else schedule
+    grp = grp if causal_group is None else causal_group
     s = fa.schedules()[sid]
     return {"id": sid, "exp_poly_every": s["emu_every"], "kv_slots": s["kv_slots"],
             "causal_group": grp if causal else None}
@@ -308,6 +310,9 @@ def run_ours(args, cfg):
                                 device_id=dev)
     import numpy as np
     import attention_forward_17_b200 as fa
+    # --schedule / --causal-group pin the kernel schedule (profiling); default: the search table
+    override = {k: v for k, v in (("schedule", args.schedule), ("causal_group", args.causal_group))
+                if v is not None}
     import seeded_inputs as si
 
     B, H, N, d = cfg["B"], cfg["H"], cfg["N"], cfg["d"]
@@ -332,7 +337,7 @@ def run_ours(args, cfg):
     # ---------------- device-resident timing, per-launch events
     for _ in range(args.warmup):
         for c in modes:
-            fa.fa_fwd(q, k, v, causal=c, out=o[c], lse=lse[c])
+            fa.fa_fwd(q, k, v, causal=c, out=o[c], lse=lse[c], **override)
     torch.cuda.synchronize()
     ev = {c: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)] for c in modes}
@@ -345,7 +350,7 @@ def run_ours(args, cfg):
         for s in range(args.steps):
             for c in modes:
                 ev[c][s][0].record(stream)
-                fa.fa_fwd(q, k, v, causal=c, out=o[c], lse=lse[c])
+                fa.fa_fwd(q, k, v, causal=c, out=o[c], lse=lse[c], **override)
                 ev[c][s][1].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -420,7 +425,8 @@ def run_ours(args, cfg):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
             "config": dict(workload_config(args.workload, cfg, world, modes),
-                           schedule={("causal" if c else "non-causal"): schedule_of(N, d, c)
+                           schedule={("causal" if c else "non-causal"):
+                                     schedule_of(N, d, c, args.schedule, args.causal_group)
                                      for c in modes}),
             "pct_of_peak": {"measured_burst": 100 * value / world / peaks["bf16"],
                             "measured_sustained": 100 * value / world / peaks["bf16_sustained"],
@@ -619,6 +625,10 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--modes", choices=sorted(MODES), default="both",
                     help="masking modes in one step (the headline uses both)")
+    ap.add_argument("--schedule", type=int, default=None,
+                    help="pin the attention kernel schedule id (default: the search table's choice)")
+    ap.add_argument("--causal-group", type=int, default=None,
+                    help="pin the causal launch group (default: the search table's choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
