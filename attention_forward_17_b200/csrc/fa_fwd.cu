@@ -43,6 +43,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceState {
     std::once_flag once;
     int status = FA_OK;   // outcome of the one-time set-up for this device
+    int sms = 0;          // streaming multiprocessors (persistent grid size)
 };
 DeviceState g_devices[kMaxDevices];
 
@@ -85,12 +86,13 @@ int device_setup(int dev) {
 // The schedule id fa_fwd uses for (N, d, causal), and the causal launch group.
 void pick_schedule(int64_t N, int64_t d, int causal, int* id, int* group) {
     const ScheduleList& list = schedules();
-    int emu = -1, slots = -1, grp = 1;
+    int emu = -1, slots = -1, grp = 1, persist = 0;
     for (const auto& e : fa::kScheduleTable)
         if (e.d == d && e.causal == (causal ? 1 : 0) && N <= e.n_max) {
             emu = e.emu;
             slots = e.slots;
             grp = e.group;
+            persist = e.persist;
             break;
         }
     int first = -1, match = -1;
@@ -98,7 +100,7 @@ void pick_schedule(int64_t N, int64_t d, int causal, int* id, int* group) {
         const fa::Schedule* s = list.items[i];
         if (s->d != d) continue;
         if (first < 0) first = i;
-        if (s->emu == emu && s->slots == slots) {
+        if (s->emu == emu && s->slots == slots && s->persist == persist) {
             match = i;
             break;
         }
@@ -107,12 +109,18 @@ void pick_schedule(int64_t N, int64_t d, int causal, int* id, int* group) {
     *group = grp > 0 ? grp : 1;
 }
 
-int current_device_ready() {
+int current_device_ready(int* sms = nullptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
     DeviceState& st = g_devices[dev];
-    std::call_once(st.once, [&] { st.status = device_setup(dev); });
+    std::call_once(st.once, [&] {
+        st.status = device_setup(dev);
+        if (st.status == FA_OK &&
+            cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            st.status = FA_ERR_CUDA;
+    });
+    if (sms) *sms = st.sms;
     return st.status;
 }
 
@@ -170,7 +178,8 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
     pick_schedule(N, d, causal, &table_id, &table_group);
     if (schedule_id < 0) schedule_id = table_id;
     if (group < 1) group = table_group;
-    if ((rc = current_device_ready()) != FA_OK) return rc;
+    int sms = 0;
+    if ((rc = current_device_ready(&sms)) != FA_OK) return rc;
     if ((rc = encoder_ready()) != FA_OK) return rc;
     const int64_t BH = B * H;
     alignas(64) CUtensorMap tq, tk, tv;
@@ -186,9 +195,14 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
     p.n_qtile = static_cast<int>((N + fa::kBlockM - 1) / fa::kBlockM);
     p.group = static_cast<int>(group < BH ? group : BH);
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-    const int64_t grid = BH * p.n_qtile;
+    int64_t grid = BH * p.n_qtile;
     if (grid > 0x7fffffffLL) return FA_ERR_SHAPE;
     const fa::Schedule* sch = list.items[schedule_id];
+    if (sch->persist) {
+        // one CTA per SM; causal work comes in units of two query tiles
+        const int64_t units = causal ? BH * ((p.n_qtile + 1) / 2) : grid;
+        grid = units < sms ? units : sms;
+    }
     const cudaError_t e = sch->launch[causal ? 1 : 0](tq, tk, tv, p, static_cast<unsigned>(grid),
                                                        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -222,13 +236,15 @@ int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float*
 
 int fa_schedule_count(void) { return schedules().count; }
 
-int fa_schedule_info(int id, int* d, int* emu_every, int* kv_slots, int* smem_bytes) {
+int fa_schedule_info(int id, int* d, int* emu_every, int* kv_slots, int* persistent,
+                     int* smem_bytes) {
     const ScheduleList& list = schedules();
     if (id < 0 || id >= list.count) return FA_ERR_ARG;
     const fa::Schedule* s = list.items[id];
     if (d) *d = s->d;
     if (emu_every) *emu_every = s->emu;
     if (kv_slots) *kv_slots = s->slots;
+    if (persistent) *persistent = s->persist;
     if (smem_bytes) *smem_bytes = s->smem_bytes;
     return FA_OK;
 }
@@ -294,6 +310,6 @@ const char* fa_strerror(int status) {
     }
 }
 
-int fa_version(void) { return (1 << 16) | 0; }
+int fa_version(void) { return (1 << 16) | 1; }
 
 }  // extern "C"

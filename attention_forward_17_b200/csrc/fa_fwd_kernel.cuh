@@ -9,7 +9,8 @@
 // products (Q K^T and P V) run on the tensor cores ("TileLang tutorial",
 // FlashAttention section).
 //
-// Blackwell mapping.  One CTA = one 128-row query tile of one (b, h) slice;
+// Blackwell mapping.  A CTA works on 128-row query tiles of (b, h) slices,
+// one per CTA or, in the persistent launch, several in turn (TileCursor);
 // 384 threads in three warpgroups:
 //   warpgroups 0 and 1  softmax.  Each warp owns 16 query rows (TMEM lanes
 //               32*quarter + 16*g ..) through the 16-lane TMEM access shapes; a
@@ -115,10 +116,12 @@ struct alignas(8) Barriers {
     uint64_t kv_full[kSlots];
     uint64_t kv_empty[kSlots];
     uint64_t q_full;            // Q tile landed in shared memory
+    uint64_t q_empty;           // every score product of the current tile done (Q reusable)
     uint64_t s_full[kSBufs];    // S_b computed
     uint64_t p_full[kSBufs];    // P_b written (and O rescaled)
     uint64_t pv_done[kSBufs];   // O += P_b V of the latest use of buffer b completed
-    uint64_t o_full;            // every product done
+    uint64_t o_full;            // every product of the current tile done
+    uint64_t o_empty;           // the epilogue has read O out of TMEM
     uint32_t tmem_base;
     volatile uint32_t abort;
 };
@@ -204,7 +207,70 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int D, bool CAUSAL, int EMU, int SLOTS>
+// The query tiles one CTA processes, in order.
+//   PERSIST = false: one tile per CTA.  Without the mask, the CTAs of one
+//     (b, h) slice are adjacent in launch order so the slice's K/V stay in L2.
+//     Under the causal mask the slices are taken `group` at a time and, inside
+//     a group, query tiles launch longest first (all the group's last tiles,
+//     then the tiles before them, ...), which keeps the group's K/V in L2
+//     while the short tiles fill the end of the grid.
+//   PERSIST = true: one CTA per SM walks several tiles, so one tile's
+//     epilogue and the next tile's Q load and first score products overlap
+//     instead of paying a CTA launch, barrier set-up and TMEM allocation per
+//     tile.  Without the mask: tiles blockIdx.x, +gridDim.x, ... in (b, h)-
+//     major order.  Under the mask: units of two tiles of one slice, qt =
+//     n-1-k then qt = k (one tile when they coincide), so every unit holds
+//     n+1 key tiles of work and a plain round-robin of units balances the
+//     CTAs; units blockIdx.x, +gridDim.x, ... in (b, h)-major order.
+template <bool CAUSAL, bool PERSIST>
+struct TileCursor {
+    int r = 0;      // round
+    int half = 0;   // causal persistent: 0 = long tile of the unit next, 1 = short tile next
+
+    __device__ __forceinline__ bool next(const FwdParams& p, int& bh, int& qt) {
+        if constexpr (!PERSIST) {
+            if (r++ > 0) return false;
+            if constexpr (CAUSAL) {
+                const int span = p.group * p.n_qtile;
+                const int g0 = (blockIdx.x / span) * p.group;
+                const int heads = min(p.group, p.BH - g0);
+                const int rr = blockIdx.x % span;
+                bh = g0 + rr % heads;
+                qt = p.n_qtile - 1 - rr / heads;
+            } else {
+                bh = blockIdx.x / p.n_qtile;
+                qt = blockIdx.x % p.n_qtile;
+            }
+            return true;
+        } else if constexpr (!CAUSAL) {
+            const int64_t i = blockIdx.x + static_cast<int64_t>(r) * gridDim.x;
+            if (i >= static_cast<int64_t>(p.BH) * p.n_qtile) return false;
+            ++r;
+            bh = static_cast<int>(i / p.n_qtile);
+            qt = static_cast<int>(i % p.n_qtile);
+            return true;
+        } else {
+            const int units = (p.n_qtile + 1) / 2;
+            const int64_t u = blockIdx.x + static_cast<int64_t>(r) * gridDim.x;
+            if (u >= static_cast<int64_t>(p.BH) * units) return false;
+            bh = static_cast<int>(u / units);
+            const int k = static_cast<int>(u % units);
+            const int hi = p.n_qtile - 1 - k;
+            if (half == 0) {
+                qt = hi;
+                if (hi == k) ++r;       // the middle tile of an odd count stands alone
+                else half = 1;
+            } else {
+                qt = k;
+                half = 0;
+                ++r;
+            }
+            return true;
+        }
+    }
+};
+
+template <int D, bool CAUSAL, int EMU, int SLOTS, bool PERSIST>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -220,35 +286,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item.  Without the mask, the CTAs of one (b, h) slice are adjacent
-    // in launch order so the slice's K/V stay in L2.  Under the causal mask the
-    // slices are taken `group` at a time and, inside a group, query tiles are
-    // launched longest first (all the group's last tiles, then the tiles before
-    // them, ...), which keeps the group's K/V in L2 while the short tiles fill
-    // the end of the grid.
-    int bh, qt;
-    if constexpr (CAUSAL) {
-        const int span = p.group * p.n_qtile;
-        const int g0 = (blockIdx.x / span) * p.group;
-        const int heads = min(p.group, p.BH - g0);
-        const int r = blockIdx.x % span;
-        bh = g0 + r % heads;
-        qt = p.n_qtile - 1 - r / heads;
-    } else {
-        bh = blockIdx.x / p.n_qtile;
-        qt = blockIdx.x % p.n_qtile;
-    }
-    const int q0 = qt * kBlockM;
     const int n_kv_all = (p.N + kBlockN - 1) / kBlockN;
-    const int n_kv = CAUSAL ? min(n_kv_all, qt + 1) : n_kv_all;
+    // keys of query tile qt: all tiles, or up to the diagonal under the mask
+    const auto kv_tiles = [&](int qt) { return CAUSAL ? min(n_kv_all, qt + 1) : n_kv_all; };
 
     const uint32_t bar_kv_full = smem_u32(&bars->kv_full[0]);
     const uint32_t bar_kv_empty = smem_u32(&bars->kv_empty[0]);
     const uint32_t bar_q_full = smem_u32(&bars->q_full);
+    const uint32_t bar_q_empty = smem_u32(&bars->q_empty);
     const uint32_t bar_s_full = smem_u32(&bars->s_full[0]);
     const uint32_t bar_p_full = smem_u32(&bars->p_full[0]);
     const uint32_t bar_pv_done = smem_u32(&bars->pv_done[0]);
     const uint32_t bar_o_full = smem_u32(&bars->o_full);
+    const uint32_t bar_o_empty = smem_u32(&bars->o_empty);
     volatile uint32_t* abort = &bars->abort;
 
     if (threadIdx.x == 0) {
@@ -257,12 +307,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar_kv_empty + 8 * s, 1);
         }
         mbar_init(bar_q_full, 1);
+        mbar_init(bar_q_empty, 1);
         for (int b = 0; b < kSBufs; ++b) {
             mbar_init(bar_s_full + 8 * b, 1);
             mbar_init(bar_p_full + 8 * b, 256);
             mbar_init(bar_pv_done + 8 * b, 1);
         }
         mbar_init(bar_o_full, 1);
+        mbar_init(bar_o_empty, 256);
         bars->abort = 0u;
         fence_barrier_init();
     }
@@ -280,6 +332,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
+    // Every role walks the same tile sequence (TileCursor).  Across tiles the
+    // score buffers and their barriers are indexed by a global step count
+    // (gs), the K/V ring by a global load count (lb = loads of earlier
+    // tiles), and the per-tile barriers (Q, O) by the tile count.
     if (warp < 8) {
         regs_increase<kRegsSoftmax>();
         // ============================================================ softmax
@@ -295,215 +351,223 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_w = static_cast<uint32_t>(L) << 16;
         const float c = p.scale_log2;
         const uint64_t c2 = f2(c, c);
-
+        TileCursor<CAUSAL, PERSIST> cur;
+        int bh, qt, gs = 0, tile = 0;
+        while (cur.next(p, bh, qt)) {
+        const int q0 = qt * kBlockM;
+        const int n_kv = kv_tiles(qt);
         float m_a = -INFINITY, m_b = -INFINITY;   // running max of c*s per row (stale by < 8)
         float l_a = 0.f, l_b = 0.f;               // fp32 sums of 2^(c*s - m) (for LSE), this thread's keys
         float lh_a = 0.f, lh_b = 0.f;             // the same weights rounded to bf16 (for O)
 
-        for (int j = 0; j < n_kv; ++j) {
-            const int bb = j % kSBufs;
-            const uint32_t t_s = tmem + lane_w + C::col_s(bb);
-            wait_bar(bar_s_full + 8 * bb, (j / kSBufs) & 1, abort, p.status);
-            tc_fence_after();
-            uint32_t s[64];
-            tmem_ld16x256b_x16(t_s, s);
-            tmem_wait_ld();
-            reg_fence64(s);
-
-            const bool masked =
-                (j * kBlockN + kBlockN > p.N) || (CAUSAL && j * kBlockN + kBlockN - 1 > q0);
-            if (masked) {
-                const int lim_a = (CAUSAL ? min(p.N, q0 + ra + 1) : p.N) - j * kBlockN;
-                const int lim_b = (CAUSAL ? min(p.N, q0 + rb + 1) : p.N) - j * kBlockN;
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int key = 8 * m + kq + e;
-                        if (key >= lim_a) s[4 * m + e] = __float_as_uint(-INFINITY);
-                        if (key >= lim_b) s[4 * m + 2 + e] = __float_as_uint(-INFINITY);
-                    }
-            }
-            // row maxima: 32 values per row in this thread, then across the 4 threads
-            float xa0 = fmaxf(__uint_as_float(s[0]), __uint_as_float(s[1]));
-            float xb0 = fmaxf(__uint_as_float(s[2]), __uint_as_float(s[3]));
-            float xa1 = fmaxf(__uint_as_float(s[4]), __uint_as_float(s[5]));
-            float xb1 = fmaxf(__uint_as_float(s[6]), __uint_as_float(s[7]));
-#pragma unroll
-            for (int m = 2; m < 16; m += 2) {
-                xa0 = max3f(xa0, __uint_as_float(s[4 * m]), __uint_as_float(s[4 * m + 1]));
-                xb0 = max3f(xb0, __uint_as_float(s[4 * m + 2]), __uint_as_float(s[4 * m + 3]));
-                xa1 = max3f(xa1, __uint_as_float(s[4 * m + 4]), __uint_as_float(s[4 * m + 5]));
-                xb1 = max3f(xb1, __uint_as_float(s[4 * m + 6]), __uint_as_float(s[4 * m + 7]));
-            }
-            float mxa = fmaxf(xa0, xa1), mxb = fmaxf(xb0, xb1);
-            mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
-            mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
-            mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
-            mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
-            const float mna = mxa * c, mnb = mxb * c;
-            const bool ga = mna > m_a + 8.0f, gb = mnb > m_b + 8.0f;
-            float alpha_a = 1.f, alpha_b = 1.f;
-            if (ga) {
-                alpha_a = ex2_approx(m_a - mna);
-                m_a = mna;
-                l_a *= alpha_a;
-                lh_a *= alpha_a;
-            }
-            if (gb) {
-                alpha_b = ex2_approx(m_b - mnb);
-                m_b = mnb;
-                l_b *= alpha_b;
-                lh_b *= alpha_b;
-            }
-            if (j > 0 && __any_sync(0xffffffffu, ga || gb)) {
-                // O holds sum_{j' < j} P V with the old reference maxima: scale
-                // these 16 rows by 2^(m_old - m_new) once the product of step
-                // j-1 has landed.
-                wait_bar(bar_pv_done + 8 * ((j - 1) % kSBufs), ((j - 1) / kSBufs) & 1, abort,
-                         p.status);
+            for (int j = 0; j < n_kv; ++j) {
+                const int gj = gs + j;                // global step: buffer and phase
+                const int bb = gj % kSBufs;
+                const uint32_t t_s = tmem + lane_w + C::col_s(bb);
+                wait_bar(bar_s_full + 8 * bb, (gj / kSBufs) & 1, abort, p.status);
                 tc_fence_after();
-                const uint32_t t_o = tmem + lane_w + C::kColO;
-                if constexpr (D == 128) {
-                    uint32_t o[64];
-                    tmem_ld16x256b_x16(t_o, o);
-                    tmem_wait_ld();
-                    reg_fence64(o);
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        o[4 * m] = __float_as_uint(__uint_as_float(o[4 * m]) * alpha_a);
-                        o[4 * m + 1] = __float_as_uint(__uint_as_float(o[4 * m + 1]) * alpha_a);
-                        o[4 * m + 2] = __float_as_uint(__uint_as_float(o[4 * m + 2]) * alpha_b);
-                        o[4 * m + 3] = __float_as_uint(__uint_as_float(o[4 * m + 3]) * alpha_b);
-                    }
-                    reg_fence64(o);
-                    tmem_st16x256b_x16(t_o, o);
-                } else {
-                    uint32_t o[32];
-                    tmem_ld16x256b_x8(t_o, o);
-                    tmem_wait_ld();
-                    reg_fence32(o);
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        o[4 * m] = __float_as_uint(__uint_as_float(o[4 * m]) * alpha_a);
-                        o[4 * m + 1] = __float_as_uint(__uint_as_float(o[4 * m + 1]) * alpha_a);
-                        o[4 * m + 2] = __float_as_uint(__uint_as_float(o[4 * m + 2]) * alpha_b);
-                        o[4 * m + 3] = __float_as_uint(__uint_as_float(o[4 * m + 3]) * alpha_b);
-                    }
-                    reg_fence32(o);
-                    tmem_st16x256b_x8(t_o, o);
+                uint32_t s[64];
+                tmem_ld16x256b_x16(t_s, s);
+                tmem_wait_ld();
+                reg_fence64(s);
+
+                const bool masked =
+                    (j * kBlockN + kBlockN > p.N) || (CAUSAL && j * kBlockN + kBlockN - 1 > q0);
+                if (masked) {
+                    const int lim_a = (CAUSAL ? min(p.N, q0 + ra + 1) : p.N) - j * kBlockN;
+                    const int lim_b = (CAUSAL ? min(p.N, q0 + rb + 1) : p.N) - j * kBlockN;
+    #pragma unroll
+                    for (int m = 0; m < 16; ++m)
+    #pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int key = 8 * m + kq + e;
+                            if (key >= lim_a) s[4 * m + e] = __float_as_uint(-INFINITY);
+                            if (key >= lim_b) s[4 * m + 2 + e] = __float_as_uint(-INFINITY);
+                        }
                 }
-            }
-            const float ua = (m_a == -INFINITY) ? 0.f : m_a;
-            const float ub = (m_b == -INFINITY) ? 0.f : m_b;
-            const uint64_t nega = f2(-ua, -ua), negb = f2(-ub, -ub);
-            // p = 2^(c*s - m) pairwise through packed FMAs; sums of the fp32
-            // weights (for LSE) and of their bf16 roundings (for O).  P word
-            // 2m / 2m+1 = keys 8m + kq + {0,1} of row a / row b, which is the
-            // 16x128b store layout at column 4m + t%4 of the P region.
-            uint64_t la2 = 0, lb2 = 0, ha2 = 0, hb2 = 0;
-            float hsa0 = 0.f, hsa1 = 0.f, hsb0 = 0.f, hsb1 = 0.f;
-            uint32_t pk[32];
-            if constexpr (FA_SOFTMAX_PHASED) {
-                // pass 1: exponents c*s - m, in place
-#pragma unroll
+                // row maxima: 32 values per row in this thread, then across the 4 threads
+                float xa0 = fmaxf(__uint_as_float(s[0]), __uint_as_float(s[1]));
+                float xb0 = fmaxf(__uint_as_float(s[2]), __uint_as_float(s[3]));
+                float xa1 = fmaxf(__uint_as_float(s[4]), __uint_as_float(s[5]));
+                float xb1 = fmaxf(__uint_as_float(s[6]), __uint_as_float(s[7]));
+    #pragma unroll
+                for (int m = 2; m < 16; m += 2) {
+                    xa0 = max3f(xa0, __uint_as_float(s[4 * m]), __uint_as_float(s[4 * m + 1]));
+                    xb0 = max3f(xb0, __uint_as_float(s[4 * m + 2]), __uint_as_float(s[4 * m + 3]));
+                    xa1 = max3f(xa1, __uint_as_float(s[4 * m + 4]), __uint_as_float(s[4 * m + 5]));
+                    xb1 = max3f(xb1, __uint_as_float(s[4 * m + 6]), __uint_as_float(s[4 * m + 7]));
+                }
+                float mxa = fmaxf(xa0, xa1), mxb = fmaxf(xb0, xb1);
+                mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
+                mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
+                mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
+                mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
+                const float mna = mxa * c, mnb = mxb * c;
+                const bool ga = mna > m_a + 8.0f, gb = mnb > m_b + 8.0f;
+                float alpha_a = 1.f, alpha_b = 1.f;
+                if (ga) {
+                    alpha_a = ex2_approx(m_a - mna);
+                    m_a = mna;
+                    l_a *= alpha_a;
+                    lh_a *= alpha_a;
+                }
+                if (gb) {
+                    alpha_b = ex2_approx(m_b - mnb);
+                    m_b = mnb;
+                    l_b *= alpha_b;
+                    lh_b *= alpha_b;
+                }
+                if (j > 0 && __any_sync(0xffffffffu, ga || gb)) {
+                    // O holds sum_{j' < j} P V with the old reference maxima: scale
+                    // these 16 rows by 2^(m_old - m_new) once the product of step
+                    // j-1 has landed.
+                    wait_bar(bar_pv_done + 8 * ((gj - 1) % kSBufs), ((gj - 1) / kSBufs) & 1, abort,
+                             p.status);
+                    tc_fence_after();
+                    const uint32_t t_o = tmem + lane_w + C::kColO;
+                    if constexpr (D == 128) {
+                        uint32_t o[64];
+                        tmem_ld16x256b_x16(t_o, o);
+                        tmem_wait_ld();
+                        reg_fence64(o);
+    #pragma unroll
+                        for (int m = 0; m < 16; ++m) {
+                            o[4 * m] = __float_as_uint(__uint_as_float(o[4 * m]) * alpha_a);
+                            o[4 * m + 1] = __float_as_uint(__uint_as_float(o[4 * m + 1]) * alpha_a);
+                            o[4 * m + 2] = __float_as_uint(__uint_as_float(o[4 * m + 2]) * alpha_b);
+                            o[4 * m + 3] = __float_as_uint(__uint_as_float(o[4 * m + 3]) * alpha_b);
+                        }
+                        reg_fence64(o);
+                        tmem_st16x256b_x16(t_o, o);
+                    } else {
+                        uint32_t o[32];
+                        tmem_ld16x256b_x8(t_o, o);
+                        tmem_wait_ld();
+                        reg_fence32(o);
+    #pragma unroll
+                        for (int m = 0; m < 8; ++m) {
+                            o[4 * m] = __float_as_uint(__uint_as_float(o[4 * m]) * alpha_a);
+                            o[4 * m + 1] = __float_as_uint(__uint_as_float(o[4 * m + 1]) * alpha_a);
+                            o[4 * m + 2] = __float_as_uint(__uint_as_float(o[4 * m + 2]) * alpha_b);
+                            o[4 * m + 3] = __float_as_uint(__uint_as_float(o[4 * m + 3]) * alpha_b);
+                        }
+                        reg_fence32(o);
+                        tmem_st16x256b_x8(t_o, o);
+                    }
+                }
+                const float ua = (m_a == -INFINITY) ? 0.f : m_a;
+                const float ub = (m_b == -INFINITY) ? 0.f : m_b;
+                const uint64_t nega = f2(-ua, -ua), negb = f2(-ub, -ub);
+                // p = 2^(c*s - m) pairwise through packed FMAs; sums of the fp32
+                // weights (for LSE) and of their bf16 roundings (for O).  P word
+                // 2m / 2m+1 = keys 8m + kq + {0,1} of row a / row b, which is the
+                // 16x128b store layout at column 4m + t%4 of the P region.
+                uint64_t la2 = 0, lb2 = 0, ha2 = 0, hb2 = 0;
+                float hsa0 = 0.f, hsa1 = 0.f, hsb0 = 0.f, hsb1 = 0.f;
+                uint32_t pk[32];
+                if constexpr (FA_SOFTMAX_PHASED) {
+                    // pass 1: exponents c*s - m, in place
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int m = i >> 1;
+                        const int o = 4 * m + 2 * (i & 1);
+                        const uint64_t x2 = fma2(f2(__uint_as_float(s[o]), __uint_as_float(s[o + 1])), c2,
+                                                 (i & 1) ? negb : nega);
+                        float x0, x1;
+                        f2_split(x2, x0, x1);
+                        s[o] = __float_as_uint(x0);
+                        s[o + 1] = __float_as_uint(x1);
+                    }
+                    // pass 2: exponentials in place
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int o = 4 * (i >> 1) + 2 * (i & 1);
+                        float p0, p1;
+                        if (EMU > 0 && (i % (EMU > 0 ? EMU : 1)) == EMU - 1) {
+                            exp2_poly2(__uint_as_float(s[o]), __uint_as_float(s[o + 1]), p0, p1);
+                        } else {
+                            p0 = ex2_approx(__uint_as_float(s[o]));
+                            p1 = ex2_approx(__uint_as_float(s[o + 1]));
+                        }
+                        s[o] = __float_as_uint(p0);
+                        s[o + 1] = __float_as_uint(p1);
+                    }
+                    // pass 3: bf16 pairs and the two sums
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int o = 4 * (i >> 1) + 2 * (i & 1);
+                        const float p0 = __uint_as_float(s[o]), p1 = __uint_as_float(s[o + 1]);
+                        const uint32_t w = pack_bf16x2(p0, p1);
+                        const uint64_t pr = f2(p0, p1);
+                        const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+                        if (i & 1) {
+                            lb2 = add2(lb2, pr);
+                            hb2 = add2(hb2, ph);
+                        } else {
+                            la2 = add2(la2, pr);
+                            ha2 = add2(ha2, ph);
+                        }
+                        pk[i] = w;
+                    }
+                } else
+    #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int m = i >> 1;
-                    const int o = 4 * m + 2 * (i & 1);
-                    const uint64_t x2 = fma2(f2(__uint_as_float(s[o]), __uint_as_float(s[o + 1])), c2,
-                                             (i & 1) ? negb : nega);
+                    const bool row_b = i & 1;
+                    const uint64_t x2 = fma2(f2(__uint_as_float(s[4 * m + 2 * row_b]),
+                                                __uint_as_float(s[4 * m + 2 * row_b + 1])),
+                                             c2, row_b ? negb : nega);
                     float x0, x1;
                     f2_split(x2, x0, x1);
-                    s[o] = __float_as_uint(x0);
-                    s[o + 1] = __float_as_uint(x1);
-                }
-                // pass 2: exponentials in place
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int o = 4 * (i >> 1) + 2 * (i & 1);
                     float p0, p1;
                     if (EMU > 0 && (i % (EMU > 0 ? EMU : 1)) == EMU - 1) {
-                        exp2_poly2(__uint_as_float(s[o]), __uint_as_float(s[o + 1]), p0, p1);
+                        exp2_poly2(x0, x1, p0, p1);
                     } else {
-                        p0 = ex2_approx(__uint_as_float(s[o]));
-                        p1 = ex2_approx(__uint_as_float(s[o + 1]));
+                        p0 = ex2_approx(x0);
+                        p1 = ex2_approx(x1);
                     }
-                    s[o] = __float_as_uint(p0);
-                    s[o + 1] = __float_as_uint(p1);
-                }
-                // pass 3: bf16 pairs and the two sums
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int o = 4 * (i >> 1) + 2 * (i & 1);
-                    const float p0 = __uint_as_float(s[o]), p1 = __uint_as_float(s[o + 1]);
                     const uint32_t w = pack_bf16x2(p0, p1);
                     const uint64_t pr = f2(p0, p1);
-                    const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-                    if (i & 1) {
-                        lb2 = add2(lb2, pr);
-                        hb2 = add2(hb2, ph);
+                    if (row_b) lb2 = add2(lb2, pr);
+                    else la2 = add2(la2, pr);
+                    if constexpr (FA_LHAT_MIXED_ADD) {
+                        if (row_b) add_bf16x2_halves(hsb0, hsb1, w);
+                        else add_bf16x2_halves(hsa0, hsa1, w);
                     } else {
-                        la2 = add2(la2, pr);
-                        ha2 = add2(ha2, ph);
+                        const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+                        if (row_b) hb2 = add2(hb2, ph);
+                        else ha2 = add2(ha2, ph);
                     }
                     pk[i] = w;
                 }
-            } else
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int m = i >> 1;
-                const bool row_b = i & 1;
-                const uint64_t x2 = fma2(f2(__uint_as_float(s[4 * m + 2 * row_b]),
-                                            __uint_as_float(s[4 * m + 2 * row_b + 1])),
-                                         c2, row_b ? negb : nega);
-                float x0, x1;
-                f2_split(x2, x0, x1);
-                float p0, p1;
-                if (EMU > 0 && (i % (EMU > 0 ? EMU : 1)) == EMU - 1) {
-                    exp2_poly2(x0, x1, p0, p1);
-                } else {
-                    p0 = ex2_approx(x0);
-                    p1 = ex2_approx(x1);
-                }
-                const uint32_t w = pack_bf16x2(p0, p1);
-                const uint64_t pr = f2(p0, p1);
-                if (row_b) lb2 = add2(lb2, pr);
-                else la2 = add2(la2, pr);
-                if constexpr (FA_LHAT_MIXED_ADD) {
-                    if (row_b) add_bf16x2_halves(hsb0, hsb1, w);
-                    else add_bf16x2_halves(hsa0, hsa1, w);
-                } else {
-                    const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-                    if (row_b) hb2 = add2(hb2, ph);
-                    else ha2 = add2(ha2, ph);
-                }
-                pk[i] = w;
+                // Pin the packed words in registers ahead of the asynchronous
+                // TMEM store.  Without this fence the multi-pass form above was
+                // observed on sm_100a to store stale register contents (the score
+                // tile) instead of P; the fence emits no instruction.
+                reg_fence32(pk);
+                tmem_st16x128b_x16(t_s + C::kColP, pk);
+                float u0, u1;
+                f2_split(la2, u0, u1);
+                l_a += u0 + u1;
+                f2_split(lb2, u0, u1);
+                l_b += u0 + u1;
+                f2_split(ha2, u0, u1);
+                lh_a += u0 + u1;
+                f2_split(hb2, u0, u1);
+                lh_b += u0 + u1;
+                lh_a += hsa0 + hsa1;
+                lh_b += hsb0 + hsb1;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_p_full + 8 * bb);
             }
-            // Pin the packed words in registers ahead of the asynchronous
-            // TMEM store.  Without this fence the multi-pass form above was
-            // observed on sm_100a to store stale register contents (the score
-            // tile) instead of P; the fence emits no instruction.
-            reg_fence32(pk);
-            tmem_st16x128b_x16(t_s + C::kColP, pk);
-            float u0, u1;
-            f2_split(la2, u0, u1);
-            l_a += u0 + u1;
-            f2_split(lb2, u0, u1);
-            l_b += u0 + u1;
-            f2_split(ha2, u0, u1);
-            lh_a += u0 + u1;
-            f2_split(hb2, u0, u1);
-            lh_b += u0 + u1;
-            lh_a += hsa0 + hsa1;
-            lh_b += hsb0 + hsb1;
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar_p_full + 8 * bb);
-        }
+        gs += n_kv;
 
         // ------------------------------------------------------------ epilogue
         // Row totals over the four threads of each row, published per tile row
-        // for the 32-lane epilogue layout (thread = row).
+        // for the 32-lane epilogue layout (thread = row); the exchange buffer
+        // alternates between tiles so a fast warp cannot overwrite values a
+        // slower partner warp has not read yet.
 #pragma unroll
         for (int sh = 1; sh <= 2; sh <<= 1) {
             l_a += __shfl_xor_sync(0xffffffffu, l_a, sh);
@@ -511,52 +575,59 @@ __global__ void __launch_bounds__(kThreads, 1)
             lh_a += __shfl_xor_sync(0xffffffffu, lh_a, sh);
             lh_b += __shfl_xor_sync(0xffffffffu, lh_b, sh);
         }
+        float* rt = red + 384 * (tile & 1);
         if ((lane & 3) == 0) {
-            red[ra] = m_a;
-            red[128 + ra] = l_a;
-            red[256 + ra] = lh_a;
-            red[rb] = m_b;
-            red[128 + rb] = l_b;
-            red[256 + rb] = lh_b;
+            rt[ra] = m_a;
+            rt[128 + ra] = l_a;
+            rt[256 + ra] = lh_a;
+            rt[rb] = m_b;
+            rt[128 + rb] = l_b;
+            rt[256 + rb] = lh_b;
         }
         named_barrier_sync(1 + quarter, 64);
         const int r = 32 * quarter + lane;        // epilogue row of this thread
         const int row = q0 + r;
-        const float m_r = red[r], l_r = red[128 + r], lh_r = red[256 + r];
-        wait_bar(bar_o_full, 0, abort, p.status);
+        const float m_r = rt[r], l_r = rt[128 + r], lh_r = rt[256 + r];
+        wait_bar(bar_o_full, tile & 1, abort, p.status);
         tc_fence_after();
+        // this thread's half of the O row, out of TMEM before anything else so
+        // the next tile's first P V product can overwrite O
+        const uint32_t t_o =
+            tmem + (static_cast<uint32_t>(32 * quarter) << 16) + C::kColO + g * (D / 2);
+        uint32_t o0[32], o1[32];
+        tmem_ld32(t_o, o0);
+        if constexpr (D == 128) tmem_ld32(t_o + 32, o1);
+        tmem_wait_ld();
+        reg_fence32(o0);
+        if constexpr (D == 128) reg_fence32(o1);
+        tc_fence_before();
+        mbar_arrive(bar_o_empty);
         const bool valid = row < p.N;
         const float inv_l = lh_r > 0.f ? 1.f / lh_r : 0.f;
         __nv_bfloat16* orow = p.o + (static_cast<int64_t>(bh) * p.N + row) * D + g * (D / 2);
-        const uint32_t t_o =
-            tmem + (static_cast<uint32_t>(32 * quarter) << 16) + C::kColO + g * (D / 2);
-#pragma unroll 1
-        for (int q = 0; q < D / 64; ++q) {
-            uint32_t o[32];
-            tmem_ld32(t_o + 32 * q, o);
-            tmem_wait_ld();
-            reg_fence32(o);
-            if (valid) {
-                uint4* dst = reinterpret_cast<uint4*>(orow + 32 * q);
+        const auto store32 = [&](const uint32_t (&o)[32], int col) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    uint4 w;
-                    w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l,
-                                      __uint_as_float(o[8 * v + 1]) * inv_l);
-                    w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l,
-                                      __uint_as_float(o[8 * v + 3]) * inv_l);
-                    w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l,
-                                      __uint_as_float(o[8 * v + 5]) * inv_l);
-                    w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l,
-                                      __uint_as_float(o[8 * v + 7]) * inv_l);
-                    dst[v] = w;
-                }
+            for (int v = 0; v < 4; ++v) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+                w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+                w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+                w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+                dst[v] = w;
             }
+        };
+        if (valid) {
+            store32(o0, 0);
+            if constexpr (D == 128) store32(o1, 32);
         }
         if (valid && g == 0) {
             float lse = l_r > 0.f ? (m_r + lg2_approx(l_r)) * 0.69314718055994531f : -INFINITY;
             if (*abort) lse = __int_as_float(0x7fc00000);
             p.lse[static_cast<int64_t>(bh) * p.N + row] = lse;
+        }
+        ++tile;
+        if (*abort) break;
         }
     } else if (warp == kProducerWarp) {
         regs_decrease<kRegsOther>();
@@ -565,12 +636,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol_q = policy_evict_first();
             const uint64_t pol_kv = policy_evict_last();
             const uint32_t slot_smem = base + C::kSlotOff;
-            mbar_arrive_expect_tx(bar_q_full, C::kTileBytes);
-#pragma unroll
-            for (int bx = 0; bx < C::kBoxes; ++bx)
-                tma_load_3d(base + C::kQOff + bx * C::kBoxBytes, &tm_q, 64 * bx, q0, bh, bar_q_full, pol_q);
-            int i = 0;
-            auto load = [&](bool is_v, int tile) {
+            int i = 0, tile = 0;
+            auto load = [&](bool is_v, int kv_tile, int bh) {
                 const int slot = i % C::kSlots;
                 const int use = i / C::kSlots;
                 if (use > 0) wait_bar(bar_kv_empty + 8 * slot, (use - 1) & 1, abort, p.status);
@@ -579,20 +646,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int bx = 0; bx < C::kBoxes; ++bx)
                     tma_load_3d(slot_smem + slot * C::kTileBytes + bx * C::kBoxBytes, map, 64 * bx,
-                                tile * kBlockN, bh, bar_kv_full + 8 * slot, pol_kv);
+                                kv_tile * kBlockN, bh, bar_kv_full + 8 * slot, pol_kv);
                 ++i;
             };
-            for (int m = 0; m < kSBufs && m < n_kv; ++m) load(false, m);
-            for (int t = 0; t < n_kv; ++t) {
-                load(true, t);
-                if (t + kSBufs < n_kv) load(false, t + kSBufs);
+            TileCursor<CAUSAL, PERSIST> cur;
+            int bh, qt;
+            while (cur.next(p, bh, qt)) {
+                const int n_kv = kv_tiles(qt);
+                // the Q buffer is free once every score product of the previous tile is done
+                if (tile > 0) wait_bar(bar_q_empty, (tile - 1) & 1, abort, p.status);
+                mbar_arrive_expect_tx(bar_q_full, C::kTileBytes);
+#pragma unroll
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                    tma_load_3d(base + C::kQOff + bx * C::kBoxBytes, &tm_q, 64 * bx, qt * kBlockM, bh,
+                                bar_q_full, pol_q);
+                for (int m = 0; m < kSBufs && m < n_kv; ++m) load(false, m, bh);
+                for (int t = 0; t < n_kv; ++t) {
+                    load(true, t, bh);
+                    if (t + kSBufs < n_kv) load(false, t + kSBufs, bh);
+                }
+                ++tile;
+                if (*abort) break;
             }
             // Every load above is waited for by an MMA issuer; in an aborted
             // CTA make sure none is still landing in shared memory at exit.
             if (*abort) {
-                for (int k = max(0, 2 * n_kv - C::kSlots); k < 2 * n_kv; ++k)
+                for (int k = max(0, i - C::kSlots); k < i; ++k)
                     wait_bar(bar_kv_full + 8 * (k % C::kSlots), (k / C::kSlots) & 1, abort, p.status);
-                wait_bar(bar_q_full, 0, abort, p.status);
+                if (tile > 0) wait_bar(bar_q_full, (tile - 1) & 1, abort, p.status);
             }
         }
         __syncwarp();
@@ -605,6 +686,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wait_bar(bar_kv_full + 8 * (i % C::kSlots), (i / C::kSlots) & 1, abort, p.status);
                 tc_fence_after();
             };
+            TileCursor<CAUSAL, PERSIST> cur;
+            int bh, qt, gs = 0, lb = 0, tile = 0;
             // Descriptors are built once; the start-address field (bits 0..13,
             // address >> 4) is advanced by plain integer adds, which never carry
             // out of the field for shared-memory addresses below 256 KiB.
@@ -615,27 +698,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                 constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false);
                 const uint64_t desc_k = smem_desc_sw128(0, 16, 1024);
                 const uint64_t a0 = desc_k + ((base + C::kQOff) >> 4);
-                wait_bar(bar_q_full, 0, abort, p.status);
-                tc_fence_after();
-                for (int m = 0; m < n_kv; ++m) {
-                    const int b = m % kSBufs;
-                    if (m >= kSBufs) {
-                        // buffer b still holds P of step m - 3 until its product is done
-                        wait_bar(bar_pv_done + 8 * b, ((m - kSBufs) / kSBufs) & 1, abort, p.status);
-                        tc_fence_after();
-                    }
-                    const int ik = load_index_k(m);
-                    wait_kv(ik);
-                    const uint64_t b0 = desc_k + (slot_addr(ik) >> 4);
-                    const uint32_t d_tmem = tmem + C::col_s(b);
+                while (cur.next(p, bh, qt)) {
+                    const int n_kv = kv_tiles(qt);
+                    wait_bar(bar_q_full, tile & 1, abort, p.status);
+                    tc_fence_after();
+                    for (int m = 0; m < n_kv; ++m) {
+                        const int gm = gs + m;
+                        const int b = gm % kSBufs;
+                        if (gm >= kSBufs) {
+                            // buffer b still holds P of step gm - 3 until its product is done
+                            wait_bar(bar_pv_done + 8 * b, ((gm - kSBufs) / kSBufs) & 1, abort, p.status);
+                            tc_fence_after();
+                        }
+                        const int ik = lb + load_index_k(m);
+                        wait_kv(ik);
+                        const uint64_t b0 = desc_k + (slot_addr(ik) >> 4);
+                        const uint32_t d_tmem = tmem + C::col_s(b);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
-                        mma_ss(d_tmem, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+                            mma_ss(d_tmem, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(bar_s_full + 8 * b);
+                        mma_commit(bar_kv_empty + 8 * (ik % C::kSlots));
                     }
-                    mma_commit(bar_s_full + 8 * b);
-                    mma_commit(bar_kv_empty + 8 * (ik % C::kSlots));
+                    mma_commit(bar_q_empty);
+                    gs += n_kv;
+                    lb += 2 * n_kv;
+                    ++tile;
+                    if (*abort) break;
                 }
+                // every score product has completed before TMEM is released
+                if (tile > 0) wait_bar(bar_q_empty, (tile - 1) & 1, abort, p.status);
             } else {
                 // ==================================================== output issuer
                 // O += P_b V: P_b from TMEM (8 columns per 16 keys); V is
@@ -644,25 +738,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // bytes per MMA.
                 constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, true);
                 const uint64_t desc_v = smem_desc_sw128(0, C::kBoxBytes, 1024);
-                for (int t = 0; t < n_kv; ++t) {
-                    const int b = t % kSBufs;
-                    const int iv = load_index_v(t, n_kv);
-                    // P_t first: it implies that every K_m (m <= t) has landed,
-                    // which the parity wait on V_t's slot relies on (see
-                    // TileCfg).
-                    wait_bar(bar_p_full + 8 * b, (t / kSBufs) & 1, abort, p.status);
-                    wait_kv(iv);
-                    const uint64_t b0 = desc_v + (slot_addr(iv) >> 4);
-                    const uint32_t a_tmem = tmem + C::col_s(b) + C::kColP;
+                while (cur.next(p, bh, qt)) {
+                    const int n_kv = kv_tiles(qt);
+                    if (tile > 0) {
+                        // O of the previous tile has been read out by the epilogue
+                        wait_bar(bar_o_empty, (tile - 1) & 1, abort, p.status);
+                        tc_fence_after();
+                    }
+                    for (int t = 0; t < n_kv; ++t) {
+                        const int gt = gs + t;
+                        const int b = gt % kSBufs;
+                        const int iv = lb + load_index_v(t, n_kv);
+                        // P_t first: it implies that every K_m (m <= t) has landed,
+                        // which the parity wait on V_t's slot relies on (see
+                        // TileCfg).
+                        wait_bar(bar_p_full + 8 * b, (gt / kSBufs) & 1, abort, p.status);
+                        wait_kv(iv);
+                        const uint64_t b0 = desc_v + (slot_addr(iv) >> 4);
+                        const uint32_t a_tmem = tmem + C::col_s(b) + C::kColP;
 #pragma unroll
-                    for (int kk = 0; kk < kBlockN / 16; ++kk)
-                        mma_ts(tmem + C::kColO, a_tmem + kk * 8, b0 + kk * (2048 >> 4), idesc_o,
-                               (t > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(bar_pv_done + 8 * b);
-                    mma_commit(bar_kv_empty + 8 * (iv % C::kSlots));
+                        for (int kk = 0; kk < kBlockN / 16; ++kk)
+                            mma_ts(tmem + C::kColO, a_tmem + kk * 8, b0 + kk * (2048 >> 4), idesc_o,
+                                   (t > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(bar_pv_done + 8 * b);
+                        mma_commit(bar_kv_empty + 8 * (iv % C::kSlots));
+                    }
+                    mma_commit(bar_o_full);
+                    gs += n_kv;
+                    lb += 2 * n_kv;
+                    ++tile;
+                    if (*abort) break;
                 }
-                mma_commit(bar_o_full);
-                wait_bar(bar_o_full, 0, abort, p.status);
+                if (tile > 0) wait_bar(bar_o_full, (tile - 1) & 1, abort, p.status);
             }
         }
         __syncwarp();

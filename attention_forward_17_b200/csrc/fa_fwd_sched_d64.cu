@@ -1,6 +1,7 @@
 // Compiled schedules of the attention kernel for head dimension 64: the
-// exponential split (EMU) times the K/V ring depth (SLOTS, 16 KiB a slot).
-// First entry = default.
+// exponential split (EMU) times the K/V ring depth (SLOTS, 16 KiB a slot),
+// plus the persistent launch for the default exponential split.  First entry
+// = default.
 #include "fa_schedules.h"
 
 namespace fa {
@@ -8,6 +9,7 @@ namespace {
 const Schedule kD64[] = {
     make_schedule<64, 4, 8>(), make_schedule<64, 0, 8>(), make_schedule<64, 2, 8>(),
     make_schedule<64, 4, 4>(), make_schedule<64, 0, 4>(), make_schedule<64, 2, 4>(),
+    make_schedule<64, 4, 8, true>(), make_schedule<64, 4, 4, true>(),
 };
 }  // namespace
 

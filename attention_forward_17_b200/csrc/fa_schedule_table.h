@@ -1,6 +1,6 @@
 // Schedule table of the attention kernel: for each head dimension, masking
 // mode and sequence-length bucket (N <= n_max), the exponential split, the
-// K/V ring depth and the causal launch group.  Written by
+// K/V ring depth, the causal launch group and the persistent launch.  Written by
 // attention_forward_17_b200/schedule_search.py on NVIDIA B200 (2026-12-02).
 #pragma once
 
@@ -15,21 +15,22 @@ struct ScheduleTableEntry {
     int emu;
     int slots;
     int group;
+    int persist;
 };
 
 constexpr ScheduleTableEntry kScheduleTable[] = {
-    {128, 0, 2048, 4, 4, 1},
-    {128, 0, 8192, 4, 4, 1},
-    {128, 0, INT64_MAX, 4, 5, 1},
-    {128, 1, 2048, 4, 4, 8},
-    {128, 1, 8192, 4, 5, 4},
-    {128, 1, INT64_MAX, 4, 5, 2},
-    {64, 0, 2048, 4, 8, 1},
-    {64, 0, 8192, 4, 8, 1},
-    {64, 0, INT64_MAX, 4, 8, 1},
-    {64, 1, 2048, 4, 4, 16},
-    {64, 1, 8192, 4, 8, 4},
-    {64, 1, INT64_MAX, 4, 4, 16},
+    {128, 0, 2048, 4, 4, 1, 1},
+    {128, 0, 8192, 4, 5, 1, 0},
+    {128, 0, INT64_MAX, 4, 5, 1, 0},
+    {128, 1, 2048, 4, 4, 1, 1},
+    {128, 1, 8192, 4, 5, 16, 0},
+    {128, 1, INT64_MAX, 4, 5, 4, 0},
+    {64, 0, 2048, 4, 4, 1, 1},
+    {64, 0, 8192, 4, 8, 1, 1},
+    {64, 0, INT64_MAX, 4, 8, 1, 1},
+    {64, 1, 2048, 4, 8, 1, 1},
+    {64, 1, 8192, 4, 4, 1, 1},
+    {64, 1, INT64_MAX, 4, 8, 8, 0},
 };
 
 }  // namespace fa

@@ -1,6 +1,6 @@
 // Registry of the compiled schedules of the attention kernel.  A schedule is
-// one instantiation of fa_fwd_kernel<D, CAUSAL, EMU, SLOTS> for both masking
-// modes; the host picks one per problem from the table the schedule search
+// one instantiation of fa_fwd_kernel<D, CAUSAL, EMU, SLOTS, PERSIST> for both
+// masking modes; the host picks one per problem from the table the schedule search
 // writes (fa_schedule_table.h) or as the caller asks (fa_fwd_schedule).
 #pragma once
 
@@ -19,6 +19,7 @@ struct Schedule {
     int d;             // head dimension
     int emu;           // every emu-th exponential pair on the FMA pipe (0 = none)
     int slots;         // K/V ring depth
+    int persist;       // 1: one CTA per SM walks several query tiles
     int smem_bytes;    // dynamic shared memory per CTA
     FwdLaunchFn launch[2];   // [causal]
     int (*setup)();          // shared-memory opt-in and register check, both modes
@@ -30,10 +31,10 @@ const Schedule* schedules_d128(int* count);
 const Schedule* schedules_d64(int* count);
 
 // Shared by both definition files.
-template <int D, bool CAUSAL, int EMU, int SLOTS>
+template <int D, bool CAUSAL, int EMU, int SLOTS, bool PERSIST>
 cudaError_t launch_schedule(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, unsigned grid, cudaStream_t stream) {
-    fa_fwd_kernel<D, CAUSAL, EMU, SLOTS>
+    fa_fwd_kernel<D, CAUSAL, EMU, SLOTS, PERSIST>
         <<<grid, kThreads, TileCfg<D, SLOTS>::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
@@ -42,9 +43,9 @@ cudaError_t launch_schedule(const CUtensorMap& tq, const CUtensorMap& tk, const 
 // was compiled with enough registers for the in-kernel warpgroup rebalance (a
 // setmaxnreg.inc asking for more than the launch allocated would never
 // return).  Returns 0 (FA_OK), -6 (FA_ERR_CUDA).
-template <int D, bool CAUSAL, int EMU, int SLOTS>
+template <int D, bool CAUSAL, int EMU, int SLOTS, bool PERSIST>
 int setup_one() {
-    auto* k = fa_fwd_kernel<D, CAUSAL, EMU, SLOTS>;
+    auto* k = fa_fwd_kernel<D, CAUSAL, EMU, SLOTS, PERSIST>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              TileCfg<D, SLOTS>::kSmemBytes) != cudaSuccess)
         return -6;
@@ -54,22 +55,24 @@ int setup_one() {
     return 0;
 }
 
-template <int D, int EMU, int SLOTS>
+template <int D, int EMU, int SLOTS, bool PERSIST>
 int setup_both() {
-    const int rc = setup_one<D, false, EMU, SLOTS>();
-    return rc ? rc : setup_one<D, true, EMU, SLOTS>();
+    const int rc = setup_one<D, false, EMU, SLOTS, PERSIST>();
+    return rc ? rc : setup_one<D, true, EMU, SLOTS, PERSIST>();
 }
 
-template <int D, int EMU, int SLOTS>
+template <int D, int EMU, int SLOTS, bool PERSIST = false>
 constexpr Schedule make_schedule() {
     static_assert(TileCfg<D, SLOTS>::kSmemBytes <= 232448, "shared memory per CTA (227 KiB)");
     static_assert(TileCfg<D, SLOTS>::kTmemCols <= 512, "tensor memory columns");
     return Schedule{D,
                     EMU,
                     SLOTS,
+                    PERSIST ? 1 : 0,
                     TileCfg<D, SLOTS>::kSmemBytes,
-                    {&launch_schedule<D, false, EMU, SLOTS>, &launch_schedule<D, true, EMU, SLOTS>},
-                    &setup_both<D, EMU, SLOTS>};
+                    {&launch_schedule<D, false, EMU, SLOTS, PERSIST>,
+                     &launch_schedule<D, true, EMU, SLOTS, PERSIST>},
+                    &setup_both<D, EMU, SLOTS, PERSIST>};
 }
 
 }  // namespace fa

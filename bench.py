@@ -286,7 +286,8 @@ def schedule_of(N, d, causal, schedule=None, causal_group=None):
     grp = grp if causal_group is None else causal_group
     s = fa.schedules()[sid]
     return {"id": sid, "exp_poly_every": s["emu_every"], "kv_slots": s["kv_slots"],
-            "causal_group": grp if causal else None}
+            "persistent": s["persistent"],
+            "causal_group": grp if (causal and not s["persistent"]) else None}
 
 
 def workload_config(name, cfg, n_gpus, modes=(False, True)):

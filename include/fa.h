@@ -97,7 +97,10 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
 /*
  * Schedules.  The kernel is compiled in several schedules: the share of
  * exponentials evaluated by polynomial on the FMA pipe instead of the
- * special-function unit, and the depth of the K/V shared-memory ring.  Under
+ * special-function unit, the depth of the K/V shared-memory ring, and the
+ * launch form (one CTA per query tile, or one persistent CTA per SM walking
+ * several tiles so that one tile's epilogue overlaps the next tile's start;
+ * under the causal mask it takes tiles in pairs of equal total work).  Under
  * the causal mask the launch order is a further runtime knob: (b, h) slices
  * are taken `causal_group` at a time, longest query tiles first within a
  * group.  fa_fwd and fa_fwd_status use, per (d, causal, N), the schedule and
@@ -108,21 +111,24 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
  *
  * fa_schedule_count - number of compiled schedules (ids 0 .. count-1).
  * fa_schedule_info  - the head dimension, exponential split (every emu_every-th
- *                     pair by polynomial; 0 = none), K/V ring depth and shared
- *                     memory per CTA of schedule `id`; FA_ERR_ARG for an
- *                     unknown id.  Output pointers may be NULL.
+ *                     pair by polynomial; 0 = none), K/V ring depth, launch
+ *                     form (1 = persistent) and shared memory per CTA of
+ *                     schedule `id`; FA_ERR_ARG for an unknown id.  Output
+ *                     pointers may be NULL.
  * fa_fwd_pick_schedule - the schedule id and causal group fa_fwd uses for
  *                     (N, d, causal).  FA_ERR_NULL, FA_ERR_SHAPE (N < 0),
  *                     FA_ERR_HEADDIM.
  * fa_fwd_schedule   - fa_fwd_status with an explicit schedule: schedule_id in
  *                     0 .. count-1 with the same d as the call, or -1 for the
  *                     table's choice; causal_group >= 1 (clamped to B*H), or 0
- *                     for the table's choice.  The arguments of fa_fwd are
+ *                     for the table's choice (the persistent launch ignores
+ *                     the group).  The arguments of fa_fwd are
  *                     checked first (same order and codes), then FA_ERR_ARG
  *                     for a bad schedule_id or causal_group.
  */
 int fa_schedule_count(void);
-int fa_schedule_info(int id, int* d, int* emu_every, int* kv_slots, int* smem_bytes);
+int fa_schedule_info(int id, int* d, int* emu_every, int* kv_slots, int* persistent,
+                     int* smem_bytes);
 int fa_fwd_pick_schedule(int64_t N, int64_t d, int causal, int* schedule_id, int* causal_group);
 int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
                     int64_t H, int64_t N, int64_t d, int causal, float scale, int schedule_id,

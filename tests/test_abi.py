@@ -35,7 +35,7 @@ def test_strerror_and_version():
         s = fa.strerror(code)
         assert isinstance(s, str) and s
     assert fa.strerror(12345) == "unknown status"
-    assert fa.version() == (1, 0)
+    assert fa.version() == (1, 1)
 
 
 def call(q=16, k=32, v=48, o=64, lse=80, B=1, H=1, N=128, d=64, causal=0, scale=0.125):
@@ -145,16 +145,18 @@ def test_schedule_registry():
     n = LIB.fa_schedule_count()
     assert n >= 2
     import ctypes
-    vals = [ctypes.c_int() for _ in range(4)]
+    vals = [ctypes.c_int() for _ in range(5)]
     seen = set()
     for i in range(n):
         assert LIB.fa_schedule_info(i, *[ctypes.byref(x) for x in vals]) == fa.FA_OK
-        d, emu, slots, smem = (x.value for x in vals)
-        assert d in (64, 128) and emu in (0, 2, 4) and slots >= 2 and 0 < smem <= 232448
-        assert (d, emu, slots) not in seen
-        seen.add((d, emu, slots))
-    assert LIB.fa_schedule_info(n, None, None, None, None) == fa.FA_ERR_ARG
-    assert LIB.fa_schedule_info(-1, None, None, None, None) == fa.FA_ERR_ARG
+        d, emu, slots, persist, smem = (x.value for x in vals)
+        assert d in (64, 128) and emu in (0, 2, 4) and slots >= 4 and persist in (0, 1)
+        assert 0 < smem <= 232448
+        assert (d, emu, slots, persist) not in seen
+        seen.add((d, emu, slots, persist))
+    assert any(k[3] == 1 for k in seen)
+    assert LIB.fa_schedule_info(n, None, None, None, None, None) == fa.FA_ERR_ARG
+    assert LIB.fa_schedule_info(-1, None, None, None, None, None) == fa.FA_ERR_ARG
     # the first schedule of each head dimension is the default
     assert fa.schedules()[0]["d"] == 128
 

@@ -1,8 +1,8 @@
 """Every compiled schedule of the attention kernel against the fp64 oracle
 (ragged N, both masking modes, wide score range), the causal launch groups
 (including a group size that does not divide B*H, so the last group is
-partial: a tile launched twice or never would show), and the table's choice
-for each problem class."""
+partial: a tile launched twice or never would show), the persistent launch
+with several tiles per CTA, and the table's choice for each problem class."""
 import numpy as np
 import pytest
 
@@ -25,7 +25,7 @@ def run_sched(qt, kt, vt, causal, sid, group):
     return pu.o_f64(o), lse.double().cpu().numpy()
 
 
-@pytest.mark.parametrize("sid", range(15))
+@pytest.mark.parametrize("sid", range(16))
 def test_every_schedule_matches_oracle(cuda_device, sid):
     sched = _schedules()
     if sid >= len(sched):
@@ -45,6 +45,22 @@ def test_causal_groups_cover_every_tile(cuda_device, group):
     o_ref, lse_ref = oracle.attention_fwd(q, k, v, True, pu.default_scale(64))
     o, lse = run_sched(qt, kt, vt, True, 9, group)
     pu.check(o, lse, o_ref, lse_ref, f"group {group}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1000, 1100])
+def test_persistent_walks_every_tile(cuda_device, d, N):
+    # 64 slices x 8 or 9 query tiles on 148 SMs: each persistent CTA takes
+    # several tiles (non-causal) or several two-tile units (causal; N = 1100
+    # gives an odd tile count, so the middle tile of each slice stands alone)
+    sched = [s for s in _schedules() if s["d"] == d and s["persistent"]]
+    assert sched, "no persistent schedule compiled"
+    (q, k, v), (qt, kt, vt) = pu.inputs(1, 64, N, d, seed=N + d)
+    for causal in (False, True):
+        o_ref, lse_ref = oracle.attention_fwd(q, k, v, causal, pu.default_scale(d))
+        for s in sched:
+            o, lse = run_sched(qt, kt, vt, causal, s["id"], 1)
+            pu.check(o, lse, o_ref, lse_ref, f"persistent {s} causal={causal} N={N}")
 
 
 def test_table_choice_is_valid():
