@@ -264,19 +264,80 @@ int fa_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, fl
     if (rc == 1) return FA_OK;
     if (rc != 0) return rc;
     if (!q_h || !k_h || !v_h || !o_h || !lse_h) return FA_ERR_NULL;
+    int sms = 0;
+    if ((rc = current_device_ready(&sms)) != FA_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t tensor_bytes = static_cast<size_t>(B * H * N * d) * 2;
-    const size_t lse_bytes = static_cast<size_t>(B * H * N) * 4;
-    if (cudaMemcpyAsync(q_d, q_h, tensor_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(k_d, k_h, tensor_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(v_d, v_h, tensor_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
-        return FA_ERR_CUDA;
-    rc = run_fwd(q_d, k_d, v_d, o_d, lse_d, B, H, N, d, causal, scale, -1, 0, nullptr, stream);
+    const int64_t BH = B * H;
+    const size_t slice = static_cast<size_t>(N * d);      // elements of one (b, h) slice
+    // Chunks of (b, h) slices, each large enough for about four waves of
+    // query tiles, at most eight: chunk c uploads while chunk c-1 computes and
+    // chunk c-2 downloads.
+    const int64_t n_qtile = (N + fa::kBlockM - 1) / fa::kBlockM;
+    int64_t per = (4 * static_cast<int64_t>(sms) + n_qtile - 1) / n_qtile;
+    if (per < 1) per = 1;
+    int64_t chunks = (BH + per - 1) / per;
+    if (chunks > 8) chunks = 8;
+    per = (BH + chunks - 1) / chunks;
+    chunks = (BH + per - 1) / per;
+    auto h2d = [&](int64_t c0, int64_t n, cudaStream_t st) {
+        const size_t off = static_cast<size_t>(c0) * slice * 2, bytes = static_cast<size_t>(n) * slice * 2;
+        return cudaMemcpyAsync(static_cast<char*>(q_d) + off, static_cast<const char*>(q_h) + off, bytes,
+                               cudaMemcpyHostToDevice, st) == cudaSuccess &&
+               cudaMemcpyAsync(static_cast<char*>(k_d) + off, static_cast<const char*>(k_h) + off, bytes,
+                               cudaMemcpyHostToDevice, st) == cudaSuccess &&
+               cudaMemcpyAsync(static_cast<char*>(v_d) + off, static_cast<const char*>(v_h) + off, bytes,
+                               cudaMemcpyHostToDevice, st) == cudaSuccess;
+    };
+    auto d2h = [&](int64_t c0, int64_t n, cudaStream_t st) {
+        const size_t off = static_cast<size_t>(c0) * slice * 2, bytes = static_cast<size_t>(n) * slice * 2;
+        return cudaMemcpyAsync(static_cast<char*>(o_h) + off, static_cast<const char*>(o_d) + off, bytes,
+                               cudaMemcpyDeviceToHost, st) == cudaSuccess &&
+               cudaMemcpyAsync(lse_h + c0 * N, lse_d + c0 * N, static_cast<size_t>(n * N) * 4,
+                               cudaMemcpyDeviceToHost, st) == cudaSuccess;
+    };
+    auto run_chunk = [&](int64_t c0, int64_t n) {
+        const size_t off = static_cast<size_t>(c0) * slice * 2;
+        return run_fwd(static_cast<const char*>(q_d) + off, static_cast<const char*>(k_d) + off,
+                       static_cast<const char*>(v_d) + off, static_cast<char*>(o_d) + off, lse_d + c0 * N,
+                       1, n, N, d, causal, scale, -1, 0, nullptr, stream);
+    };
+    if (chunks <= 1) {
+        if (!h2d(0, BH, s)) return FA_ERR_CUDA;
+        if ((rc = run_chunk(0, BH)) != FA_OK) return rc;
+        return d2h(0, BH, s) ? FA_OK : FA_ERR_CUDA;
+    }
+    // Copies run on two streams of their own, ordered against `stream` by
+    // events; `stream` waits for the last download, so its completion still
+    // means the whole call is done.  Streams and events are released by the
+    // runtime once their work has completed.
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[2 * 8 + 2] = {};
+    const int n_ev = static_cast<int>(2 * chunks + 2);
+    bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess;
+    for (int i = 0; ok && i < n_ev; ++i)
+        ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+    cudaEvent_t ev_start = ev[0], ev_done = ev[1];
+    ok = ok && cudaEventRecord(ev_start, s) == cudaSuccess &&
+         cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
+         cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess;
+    for (int64_t c = 0; ok && c < chunks; ++c) {
+        const int64_t c0 = c * per, n = (c0 + per <= BH) ? per : BH - c0;
+        cudaEvent_t ev_in = ev[2 + 2 * c], ev_k = ev[3 + 2 * c];
+        ok = h2d(c0, n, s_in) && cudaEventRecord(ev_in, s_in) == cudaSuccess &&
+             cudaStreamWaitEvent(s, ev_in, 0) == cudaSuccess;
+        if (ok && (rc = run_chunk(c0, n)) != FA_OK) break;
+        ok = ok && cudaEventRecord(ev_k, s) == cudaSuccess &&
+             cudaStreamWaitEvent(s_out, ev_k, 0) == cudaSuccess && d2h(c0, n, s_out);
+    }
+    ok = ok && rc == FA_OK && cudaEventRecord(ev_done, s_out) == cudaSuccess &&
+         cudaStreamWaitEvent(s, ev_done, 0) == cudaSuccess;
+    for (int i = 0; i < n_ev; ++i)
+        if (ev[i]) cudaEventDestroy(ev[i]);
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
     if (rc != FA_OK) return rc;
-    if (cudaMemcpyAsync(o_h, o_d, tensor_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(lse_h, lse_d, lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return FA_ERR_CUDA;
-    return FA_OK;
+    return ok ? FA_OK : FA_ERR_CUDA;
 }
 
 int fa_selftest_wait_timeout(int* dev_status, int64_t limit_us, int arrive, void* stream) {

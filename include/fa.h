@@ -137,13 +137,19 @@ int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float*
 /*
  * fa_fwd_host - the same computation starting from and ending in host memory.
  *
- * Enqueues on `stream`: copies q_h, k_h, v_h (host, bf16 [B,H,N,d]; pinned
- * memory makes the copies asynchronous) into the caller's device buffers q_d,
- * k_d, v_d; runs fa_fwd on them into o_d and lse_d; copies o_d and lse_d back
- * into o_h and lse_h (host).  Nothing is allocated; the call returns without
- * synchronising, so the host buffers must stay valid until the stream has
- * completed.  Argument checks are those of fa_fwd applied to the device
- * buffers, plus FA_ERR_NULL for a NULL host pointer.
+ * Copies q_h, k_h, v_h (host, bf16 [B,H,N,d]; pinned memory makes the copies
+ * asynchronous) into the caller's device buffers q_d, k_d, v_d; runs the
+ * forward pass on them into o_d and lse_d; copies o_d and lse_d back into o_h
+ * and lse_h (host).  The (b, h) slices are processed in up to eight chunks so
+ * that uploads, kernels and downloads of consecutive chunks overlap: the
+ * kernels run on `stream`, the copies on two streams the call creates and
+ * releases (the runtime frees them once their work is done), ordered by
+ * events so that the copies start after all earlier work on `stream` and
+ * `stream` completes only after the last download.  Nothing is allocated on
+ * the device; the call returns without synchronising, so the host buffers must
+ * stay valid until `stream` has completed.  Argument checks are those of
+ * fa_fwd applied to the device buffers, plus FA_ERR_NULL for a NULL host
+ * pointer; a failure after some work was enqueued returns FA_ERR_CUDA.
  */
 int fa_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, float* lse_h,
                 void* q_d, void* k_d, void* v_d, void* o_d, float* lse_d, int64_t B, int64_t H,

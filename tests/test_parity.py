@@ -191,6 +191,35 @@ def test_host_entry_matches_device_entry(cuda_device):
     assert torch.equal(o_h, o_dev.cpu()) and torch.equal(l_h, l_dev.cpu())
 
 
+@pytest.mark.parametrize("B,H,N,d", [(2, 32, 2048, 64), (3, 7, 4096, 128), (1, 250, 640, 64)])
+def test_host_entry_pipelined_chunks(cuda_device, B, H, N, d):
+    # enough (b, h) slices that the host entry splits them into several chunks
+    # (uploads, kernels and downloads on different streams); a ragged last chunk
+    # in the second and third cases.  Must equal the device entry bit for bit,
+    # also when the stream already holds other work, and match sampled oracle rows.
+    import torch
+    import attention_forward_17_b200 as fa
+    (q, k, v), (qt, kt, vt) = pu.inputs(B, H, N, d, seed=B + H + N)
+    q_h, k_h, v_h = (t.cpu().pin_memory() for t in (qt, kt, vt))
+    o_h = torch.empty_like(q_h).pin_memory()
+    l_h = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    q_d, k_d, v_d, o_d = (torch.zeros_like(qt) for _ in range(4))
+    l_d = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    for causal in (False, True):
+        o_dev, l_dev = pu.run(qt, kt, vt, causal)
+        o_h.zero_()
+        busy = torch.randn(4096, 4096, device="cuda")
+        busy = busy @ busy                      # queued work ahead of the call on the same stream
+        fa.fa_fwd_host(q_h, k_h, v_h, o_h, l_h, q_d, k_d, v_d, o_d, l_d, causal=causal)
+        torch.cuda.current_stream().synchronize()
+        assert torch.equal(o_h, o_dev.cpu()) and torch.equal(l_h, l_dev.cpu()), f"causal={causal}"
+        rows = pu.sample_rows(B, H, N, 48, seed=N)
+        o_ref, l_ref = oracle.attention_rows(q, k, v, causal, pu.default_scale(d), rows)
+        o_g = pu.o_f64(o_h).reshape(-1, d)[rows]
+        l_g = l_h.double().numpy().reshape(-1)[rows]
+        pu.check(o_g, l_g, o_ref, l_ref, f"host entry B={B} H={H} N={N} d={d} causal={causal}")
+
+
 def test_status_word_stays_clear(cuda_device):
     import torch
     import attention_forward_17_b200 as fa
