@@ -198,7 +198,7 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
     int64_t grid = BH * p.n_qtile;
     if (grid > 0x7fffffffLL) return FA_ERR_SHAPE;
     const fa::Schedule* sch = list.items[schedule_id];
-    if (sch->persist) {
+    if (sch->persist == 1) {
         // one CTA per SM; causal work comes in units of two query tiles
         const int64_t units = causal ? BH * ((p.n_qtile + 1) / 2) : grid;
         grid = units < sms ? units : sms;

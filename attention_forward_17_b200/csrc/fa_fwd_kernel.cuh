@@ -112,7 +112,8 @@ struct TileCfg {
 };
 
 template <int kSlots>
-struct alignas(8) Barriers {
+struct alignas(16) Barriers {
+    uint32_t clc_resp[2][4];    // cluster-launch-control responses (16-byte aligned)
     uint64_t kv_full[kSlots];
     uint64_t kv_empty[kSlots];
     uint64_t q_full;            // Q tile landed in shared memory
@@ -122,6 +123,8 @@ struct alignas(8) Barriers {
     uint64_t pv_done[kSBufs];   // O += P_b V of the latest use of buffer b completed
     uint64_t o_full;            // every product of the current tile done
     uint64_t o_empty;           // the epilogue has read O out of TMEM
+    uint64_t clc_full[2];       // response of a cancellation request landed
+    uint64_t clc_empty[2];      // every role has read that response
     uint32_t tmem_base;
     volatile uint32_t abort;
 };
@@ -208,39 +211,98 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
 
 // ---------------------------------------------------------------- the kernel
 // The query tiles one CTA processes, in order.
-//   PERSIST = false: one tile per CTA.  Without the mask, the CTAs of one
-//     (b, h) slice are adjacent in launch order so the slice's K/V stay in L2.
-//     Under the causal mask the slices are taken `group` at a time and, inside
-//     a group, query tiles launch longest first (all the group's last tiles,
+//   PERSIST = 0: one tile per CTA.  Without the mask, the CTAs of one (b, h)
+//     slice are adjacent in launch order so the slice's K/V stay in L2.  Under
+//     the causal mask the slices are taken `group` at a time and, inside a
+//     group, query tiles launch longest first (all the group's last tiles,
 //     then the tiles before them, ...), which keeps the group's K/V in L2
 //     while the short tiles fill the end of the grid.
-//   PERSIST = true: one CTA per SM walks several tiles, so one tile's
-//     epilogue and the next tile's Q load and first score products overlap
-//     instead of paying a CTA launch, barrier set-up and TMEM allocation per
-//     tile.  Without the mask: tiles blockIdx.x, +gridDim.x, ... in (b, h)-
-//     major order.  Under the mask: units of two tiles of one slice, qt =
-//     n-1-k then qt = k (one tile when they coincide), so every unit holds
-//     n+1 key tiles of work and a plain round-robin of units balances the
-//     CTAs; units blockIdx.x, +gridDim.x, ... in (b, h)-major order.
-template <bool CAUSAL, bool PERSIST>
-struct TileCursor {
-    int r = 0;      // round
-    int half = 0;   // causal persistent: 0 = long tile of the unit next, 1 = short tile next
+//   PERSIST = 1: one CTA per SM walks several tiles, so one tile's epilogue
+//     and the next tile's Q load and first score products overlap instead of
+//     paying a CTA launch, barrier set-up and TMEM allocation per tile.
+//     Without the mask: tiles blockIdx.x, +gridDim.x, ... in (b, h)-major
+//     order.  Under the mask: units of two tiles of one slice, qt = n-1-k then
+//     qt = k (one tile when they coincide), so every unit holds n+1 key tiles
+//     of work and a plain round-robin of units balances the CTAs.
+//   PERSIST = 2: the grid and tile order of PERSIST = 0, but a CTA that is
+//     about to finish a tile asks the scheduler (cluster launch control) to
+//     cancel the next CTA that has not launched yet and takes over its tile,
+//     so tiles overlap as in PERSIST = 1 while the hardware's launch order and
+//     dynamic balance are kept.  The producer issues the request; every role
+//     reads the response from one of two shared-memory slots (full / empty
+//     mbarriers).  After the first refusal no further request is made.
+template <bool CAUSAL>
+__device__ __forceinline__ void map_tile(const FwdParams& p, int id, int& bh, int& qt) {
+    if constexpr (CAUSAL) {
+        const int span = p.group * p.n_qtile;
+        const int g0 = (id / span) * p.group;
+        const int heads = min(p.group, p.BH - g0);
+        const int rr = id % span;
+        bh = g0 + rr % heads;
+        qt = p.n_qtile - 1 - rr / heads;
+    } else {
+        bh = id / p.n_qtile;
+        qt = id % p.n_qtile;
+    }
+}
 
-    __device__ __forceinline__ bool next(const FwdParams& p, int& bh, int& qt) {
-        if constexpr (!PERSIST) {
-            if (r++ > 0) return false;
-            if constexpr (CAUSAL) {
-                const int span = p.group * p.n_qtile;
-                const int g0 = (blockIdx.x / span) * p.group;
-                const int heads = min(p.group, p.BH - g0);
-                const int rr = blockIdx.x % span;
-                bh = g0 + rr % heads;
-                qt = p.n_qtile - 1 - rr / heads;
-            } else {
-                bh = blockIdx.x / p.n_qtile;
-                qt = blockIdx.x % p.n_qtile;
+constexpr int kClcReaders = 11;   // 8 softmax warps, producer, two MMA issuers
+
+template <bool CAUSAL, int PERSIST>
+struct TileCursor {
+    int r = 0;      // tiles handed out so far
+    int half = 0;   // PERSIST 1, causal: 0 = long tile of the unit next, 1 = short tile next
+    bool done = false;
+    // PERSIST 2
+    uint32_t resp = 0, full = 0, empty = 0;   // slot 0 addresses (slot 1: +16 / +8 / +8)
+    volatile uint32_t* abort = nullptr;
+    int* status = nullptr;
+
+    // The producer's request for the tile after the current one.
+    __device__ __forceinline__ void request() {
+        if constexpr (PERSIST == 2) {
+            if (done || *abort) {
+                done = true;
+                return;
             }
+            const int q = r - 1, slot = q & 1, use = q >> 1;
+            if (use > 0) wait_bar(empty + 8 * slot, (use - 1) & 1, abort, status);
+            mbar_arrive_expect_tx(full + 8 * slot, 16);
+            clc_try_cancel(resp + 16 * slot, full + 8 * slot);
+        }
+    }
+
+    // WARP: called by all 32 lanes of a warp (one arrival for the warp).
+    template <bool WARP>
+    __device__ __forceinline__ bool next(const FwdParams& p, int& bh, int& qt) {
+        if constexpr (PERSIST == 0) {
+            if (r++ > 0) return false;
+            map_tile<CAUSAL>(p, blockIdx.x, bh, qt);
+            return true;
+        } else if constexpr (PERSIST == 2) {
+            if (r == 0) {
+                ++r;
+                map_tile<CAUSAL>(p, blockIdx.x, bh, qt);
+                return true;
+            }
+            if (done) return false;
+            const int q = r - 1, slot = q & 1, use = q >> 1;
+            const uint32_t fb = full + 8 * slot;
+            wait_bar(fb, use & 1, abort, status);
+            uint32_t x = 0;
+            const bool got = mbar_try_wait(fb, use & 1) && clc_query(resp + 16 * slot, x);
+            if constexpr (WARP) {
+                __syncwarp();
+                if ((threadIdx.x & 31) == 0) mbar_arrive(empty + 8 * slot);
+            } else {
+                mbar_arrive(empty + 8 * slot);
+            }
+            if (!got || static_cast<int64_t>(x) >= static_cast<int64_t>(p.BH) * p.n_qtile) {
+                done = true;
+                return false;
+            }
+            ++r;
+            map_tile<CAUSAL>(p, static_cast<int>(x), bh, qt);
             return true;
         } else if constexpr (!CAUSAL) {
             const int64_t i = blockIdx.x + static_cast<int64_t>(r) * gridDim.x;
@@ -270,7 +332,7 @@ struct TileCursor {
     }
 };
 
-template <int D, bool CAUSAL, int EMU, int SLOTS, bool PERSIST>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int PERSIST>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -300,6 +362,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_o_full = smem_u32(&bars->o_full);
     const uint32_t bar_o_empty = smem_u32(&bars->o_empty);
     volatile uint32_t* abort = &bars->abort;
+    const auto make_cursor = [&]() {
+        TileCursor<CAUSAL, PERSIST> c;
+        c.resp = smem_u32(&bars->clc_resp[0][0]);
+        c.full = smem_u32(&bars->clc_full[0]);
+        c.empty = smem_u32(&bars->clc_empty[0]);
+        c.abort = abort;
+        c.status = p.status;
+        return c;
+    };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kSlots; ++s) {
@@ -315,6 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(bar_o_full, 1);
         mbar_init(bar_o_empty, 256);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&bars->clc_full[i]), 1);
+            mbar_init(smem_u32(&bars->clc_empty[i]), kClcReaders);
+        }
         bars->abort = 0u;
         fence_barrier_init();
     }
@@ -351,9 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_w = static_cast<uint32_t>(L) << 16;
         const float c = p.scale_log2;
         const uint64_t c2 = f2(c, c);
-        TileCursor<CAUSAL, PERSIST> cur;
+        auto cur = make_cursor();
         int bh, qt, gs = 0, tile = 0;
-        while (cur.next(p, bh, qt)) {
+        while (cur.template next<true>(p, bh, qt)) {
         const int q0 = qt * kBlockM;
         const int n_kv = kv_tiles(qt);
         float m_a = -INFINITY, m_b = -INFINITY;   // running max of c*s per row (stale by < 8)
@@ -649,9 +724,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 kv_tile * kBlockN, bh, bar_kv_full + 8 * slot, pol_kv);
                 ++i;
             };
-            TileCursor<CAUSAL, PERSIST> cur;
+            auto cur = make_cursor();
             int bh, qt;
-            while (cur.next(p, bh, qt)) {
+            while (cur.template next<false>(p, bh, qt)) {
                 const int n_kv = kv_tiles(qt);
                 // the Q buffer is free once every score product of the previous tile is done
                 if (tile > 0) wait_bar(bar_q_empty, (tile - 1) & 1, abort, p.status);
@@ -665,8 +740,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     load(true, t, bh);
                     if (t + kSBufs < n_kv) load(false, t + kSBufs, bh);
                 }
+                // PERSIST 2: claim the next tile now that this one's loads are queued
+                // (after an abort the request is skipped and the cursor ends)
+                cur.request();
                 ++tile;
-                if (*abort) break;
+                if (PERSIST != 2 && *abort) break;
             }
             // Every load above is waited for by an MMA issuer; in an aborted
             // CTA make sure none is still landing in shared memory at exit.
@@ -686,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wait_bar(bar_kv_full + 8 * (i % C::kSlots), (i / C::kSlots) & 1, abort, p.status);
                 tc_fence_after();
             };
-            TileCursor<CAUSAL, PERSIST> cur;
+            auto cur = make_cursor();
             int bh, qt, gs = 0, lb = 0, tile = 0;
             // Descriptors are built once; the start-address field (bits 0..13,
             // address >> 4) is advanced by plain integer adds, which never carry
@@ -698,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false);
                 const uint64_t desc_k = smem_desc_sw128(0, 16, 1024);
                 const uint64_t a0 = desc_k + ((base + C::kQOff) >> 4);
-                while (cur.next(p, bh, qt)) {
+                while (cur.template next<false>(p, bh, qt)) {
                     const int n_kv = kv_tiles(qt);
                     wait_bar(bar_q_full, tile & 1, abort, p.status);
                     tc_fence_after();
@@ -738,7 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // bytes per MMA.
                 constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, true);
                 const uint64_t desc_v = smem_desc_sw128(0, C::kBoxBytes, 1024);
-                while (cur.next(p, bh, qt)) {
+                while (cur.template next<false>(p, bh, qt)) {
                     const int n_kv = kv_tiles(qt);
                     if (tile > 0) {
                         // O of the previous tile has been read out by the epilogue

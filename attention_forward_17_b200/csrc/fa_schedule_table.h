@@ -19,18 +19,18 @@ struct ScheduleTableEntry {
 };
 
 constexpr ScheduleTableEntry kScheduleTable[] = {
-    {128, 0, 2048, 4, 4, 1, 1},
+    {128, 0, 2048, 4, 4, 1, 2},
     {128, 0, 8192, 4, 5, 1, 0},
     {128, 0, INT64_MAX, 4, 5, 1, 0},
     {128, 1, 2048, 4, 4, 1, 1},
     {128, 1, 8192, 4, 5, 16, 0},
     {128, 1, INT64_MAX, 4, 5, 4, 0},
-    {64, 0, 2048, 4, 4, 1, 1},
-    {64, 0, 8192, 4, 8, 1, 1},
-    {64, 0, INT64_MAX, 4, 8, 1, 1},
+    {64, 0, 2048, 4, 8, 1, 2},
+    {64, 0, 8192, 4, 8, 1, 2},
+    {64, 0, INT64_MAX, 4, 8, 1, 0},
     {64, 1, 2048, 4, 8, 1, 1},
-    {64, 1, 8192, 4, 4, 1, 1},
-    {64, 1, INT64_MAX, 4, 8, 8, 0},
+    {64, 1, 8192, 4, 8, 16, 2},
+    {64, 1, INT64_MAX, 4, 8, 16, 0},
 };
 
 }  // namespace fa

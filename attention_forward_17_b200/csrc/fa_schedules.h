@@ -19,7 +19,8 @@ struct Schedule {
     int d;             // head dimension
     int emu;           // every emu-th exponential pair on the FMA pipe (0 = none)
     int slots;         // K/V ring depth
-    int persist;       // 1: one CTA per SM walks several query tiles
+    int persist;       // launch form: 0 one tile per CTA, 1 persistent (static), 2 persistent by
+                       // cluster launch control (tiles taken over from unlaunched CTAs)
     int smem_bytes;    // dynamic shared memory per CTA
     FwdLaunchFn launch[2];   // [causal]
     int (*setup)();          // shared-memory opt-in and register check, both modes
@@ -31,7 +32,7 @@ const Schedule* schedules_d128(int* count);
 const Schedule* schedules_d64(int* count);
 
 // Shared by both definition files.
-template <int D, bool CAUSAL, int EMU, int SLOTS, bool PERSIST>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int PERSIST>
 cudaError_t launch_schedule(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, unsigned grid, cudaStream_t stream) {
     fa_fwd_kernel<D, CAUSAL, EMU, SLOTS, PERSIST>
@@ -43,7 +44,7 @@ cudaError_t launch_schedule(const CUtensorMap& tq, const CUtensorMap& tk, const 
 // was compiled with enough registers for the in-kernel warpgroup rebalance (a
 // setmaxnreg.inc asking for more than the launch allocated would never
 // return).  Returns 0 (FA_OK), -6 (FA_ERR_CUDA).
-template <int D, bool CAUSAL, int EMU, int SLOTS, bool PERSIST>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int PERSIST>
 int setup_one() {
     auto* k = fa_fwd_kernel<D, CAUSAL, EMU, SLOTS, PERSIST>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -55,20 +56,20 @@ int setup_one() {
     return 0;
 }
 
-template <int D, int EMU, int SLOTS, bool PERSIST>
+template <int D, int EMU, int SLOTS, int PERSIST>
 int setup_both() {
     const int rc = setup_one<D, false, EMU, SLOTS, PERSIST>();
     return rc ? rc : setup_one<D, true, EMU, SLOTS, PERSIST>();
 }
 
-template <int D, int EMU, int SLOTS, bool PERSIST = false>
+template <int D, int EMU, int SLOTS, int PERSIST = 0>
 constexpr Schedule make_schedule() {
     static_assert(TileCfg<D, SLOTS>::kSmemBytes <= 232448, "shared memory per CTA (227 KiB)");
     static_assert(TileCfg<D, SLOTS>::kTmemCols <= 512, "tensor memory columns");
     return Schedule{D,
                     EMU,
                     SLOTS,
-                    PERSIST ? 1 : 0,
+                    PERSIST,
                     TileCfg<D, SLOTS>::kSmemBytes,
                     {&launch_schedule<D, false, EMU, SLOTS, PERSIST>,
                      &launch_schedule<D, true, EMU, SLOTS, PERSIST>},

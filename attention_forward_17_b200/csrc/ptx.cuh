@@ -94,6 +94,34 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     return p;
 }
 
+// ------------------------------------------------------------------ cluster launch control
+// Asks the scheduler to cancel one CTA of this grid that has not launched yet
+// (its work then belongs to the caller).  The 16-byte response lands in shared
+// memory at `resp` and completes 16 transaction bytes on the mbarrier.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+    asm volatile(
+        "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];"
+        ::"r"(resp), "r"(bar)
+        : "memory");
+}
+
+// Decodes a response: true and the cancelled CTA's x index, or false when no
+// CTA was left to cancel.
+__device__ __forceinline__ bool clc_query(uint32_t resp, uint32_t& ctaid_x) {
+    uint32_t canceled, x;
+    asm volatile(
+        "{\n\t.reg .b128 rr;\n\t.reg .pred p;\n\t"
+        "ld.shared.b128 rr, [%2];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, rr;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t"
+        "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, rr;\n\t}"
+        : "=r"(canceled), "=r"(x)
+        : "r"(resp)
+        : "memory");
+    ctaid_x = x;
+    return canceled != 0;
+}
+
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),

@@ -4,11 +4,13 @@ benchmark and validate every candidate, cache the winner).
 
 The search space is what libfa_b200.so has compiled (``schedules()``): the
 share of exponentials evaluated by polynomial on the FMA pipe (none, 1/4, 1/2)
-times the depth of the K/V shared-memory ring, plus the persistent launch (one
-CTA per SM walking several query tiles), each instantiation already filtered
-at compile time to fit 227 KiB of shared memory and 512 TMEM columns.  Under
-the causal mask the launch-group size (heads whose query tiles are launched
-longest-first together) of the one-tile-per-CTA launch is searched as well.
+times the depth of the K/V shared-memory ring, plus two persistent launch
+forms (one CTA per SM walking several query tiles; or one CTA per tile whose
+running CTAs take over the tiles of unlaunched ones by cluster launch
+control), each instantiation already filtered at compile time to fit 227 KiB
+of shared memory and 512 TMEM columns.  Under the causal mask the launch-group
+size (heads whose query tiles are launched longest-first together) is searched
+as well, for the launch forms that follow the grid order.
 
 For every head dimension, masking mode and sequence-length bucket the script
 times each candidate on a B200 (CUDA events, inputs larger than L2), checks
@@ -87,7 +89,7 @@ def search(log=print):
                 o = torch.empty_like(ref_o)
                 lse = torch.empty_like(ref_l)
                 groups = [g for g in GROUPS if g <= B * H] if causal else [1]
-                cand = [(s, g) for s in cands for g in (groups if not s["persistent"] else [1])]
+                cand = [(s, g) for s in cands for g in (groups if s["persistent"] != 1 else [1])]
                 # validate each candidate once against the default schedule's output
                 valid = []
                 for s, g in cand:

@@ -287,7 +287,7 @@ def schedule_of(N, d, causal, schedule=None, causal_group=None):
     s = fa.schedules()[sid]
     return {"id": sid, "exp_poly_every": s["emu_every"], "kv_slots": s["kv_slots"],
             "persistent": s["persistent"],
-            "causal_group": grp if (causal and not s["persistent"]) else None}
+            "causal_group": grp if (causal and s["persistent"] != 1) else None}
 
 
 def workload_config(name, cfg, n_gpus, modes=(False, True)):

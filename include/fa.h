@@ -98,9 +98,11 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
  * Schedules.  The kernel is compiled in several schedules: the share of
  * exponentials evaluated by polynomial on the FMA pipe instead of the
  * special-function unit, the depth of the K/V shared-memory ring, and the
- * launch form (one CTA per query tile, or one persistent CTA per SM walking
- * several tiles so that one tile's epilogue overlaps the next tile's start;
- * under the causal mask it takes tiles in pairs of equal total work).  Under
+ * launch form (one CTA per query tile; one persistent CTA per SM walking
+ * several tiles so that one tile's epilogue overlaps the next tile's start,
+ * under the causal mask in pairs of tiles of equal total work; or one CTA per
+ * tile where a running CTA takes over the tiles of CTAs that have not launched
+ * yet).  Under
  * the causal mask the launch order is a further runtime knob: (b, h) slices
  * are taken `causal_group` at a time, longest query tiles first within a
  * group.  fa_fwd and fa_fwd_status use, per (d, causal, N), the schedule and
@@ -112,7 +114,10 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
  * fa_schedule_count - number of compiled schedules (ids 0 .. count-1).
  * fa_schedule_info  - the head dimension, exponential split (every emu_every-th
  *                     pair by polynomial; 0 = none), K/V ring depth, launch
- *                     form (1 = persistent) and shared memory per CTA of
+ *                     form (0 = one CTA per query tile, 1 = persistent with a
+ *                     static tile assignment, 2 = one CTA per tile whose
+ *                     running CTAs take over the tiles of CTAs not launched
+ *                     yet, through cluster launch control) and shared memory per CTA of
  *                     schedule `id`; FA_ERR_ARG for an unknown id.  Output
  *                     pointers may be NULL.
  * fa_fwd_pick_schedule - the schedule id and causal group fa_fwd uses for
@@ -121,8 +126,8 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
  * fa_fwd_schedule   - fa_fwd_status with an explicit schedule: schedule_id in
  *                     0 .. count-1 with the same d as the call, or -1 for the
  *                     table's choice; causal_group >= 1 (clamped to B*H), or 0
- *                     for the table's choice (the persistent launch ignores
- *                     the group).  The arguments of fa_fwd are
+ *                     for the table's choice (the static persistent launch
+ *                     ignores the group).  The arguments of fa_fwd are
  *                     checked first (same order and codes), then FA_ERR_ARG
  *                     for a bad schedule_id or causal_group.
  */

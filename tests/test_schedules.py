@@ -25,7 +25,7 @@ def run_sched(qt, kt, vt, causal, sid, group):
     return pu.o_f64(o), lse.double().cpu().numpy()
 
 
-@pytest.mark.parametrize("sid", range(16))
+@pytest.mark.parametrize("sid", range(24))
 def test_every_schedule_matches_oracle(cuda_device, sid):
     sched = _schedules()
     if sid >= len(sched):
@@ -43,8 +43,10 @@ def test_causal_groups_cover_every_tile(cuda_device, group):
     # B*H = 5 slices of 5 query tiles (N = 600, last tile ragged)
     (q, k, v), (qt, kt, vt) = pu.inputs(1, 5, 600, 64, seed=group)
     o_ref, lse_ref = oracle.attention_fwd(q, k, v, True, pu.default_scale(64))
-    o, lse = run_sched(qt, kt, vt, True, 9, group)
-    pu.check(o, lse, o_ref, lse_ref, f"group {group}")
+    for s in _schedules():
+        if s["d"] == 64 and s["persistent"] != 1:      # the launch forms that use the group
+            o, lse = run_sched(qt, kt, vt, True, s["id"], group)
+            pu.check(o, lse, o_ref, lse_ref, f"group {group} schedule {s}")
 
 
 @pytest.mark.parametrize("d", [64, 128])
@@ -52,7 +54,9 @@ def test_causal_groups_cover_every_tile(cuda_device, group):
 def test_persistent_walks_every_tile(cuda_device, d, N):
     # 64 slices x 8 or 9 query tiles on 148 SMs: each persistent CTA takes
     # several tiles (non-causal) or several two-tile units (causal; N = 1100
-    # gives an odd tile count, so the middle tile of each slice stands alone)
+    # gives an odd tile count, so the middle tile of each slice stands alone);
+    # with cluster launch control, CTAs take over the tiles of CTAs that had not
+    # launched yet
     sched = [s for s in _schedules() if s["d"] == d and s["persistent"]]
     assert sched, "no persistent schedule compiled"
     (q, k, v), (qt, kt, vt) = pu.inputs(1, 64, N, d, seed=N + d)
