@@ -86,13 +86,14 @@ int device_setup(int dev) {
 // The schedule id fa_fwd uses for (N, d, causal), and the causal launch group.
 void pick_schedule(int64_t N, int64_t d, int causal, int* id, int* group) {
     const ScheduleList& list = schedules();
-    int emu = -1, slots = -1, grp = 1, persist = 0;
+    int emu = -1, slots = -1, grp = 1, persist = 0, alg = 0;
     for (const auto& e : fa::kScheduleTable)
         if (e.d == d && e.causal == (causal ? 1 : 0) && N <= e.n_max) {
             emu = e.emu;
             slots = e.slots;
             grp = e.group;
             persist = e.persist;
+            alg = e.alg;
             break;
         }
     int first = -1, match = -1;
@@ -100,7 +101,7 @@ void pick_schedule(int64_t N, int64_t d, int causal, int* id, int* group) {
         const fa::Schedule* s = list.items[i];
         if (s->d != d) continue;
         if (first < 0) first = i;
-        if (s->emu == emu && s->slots == slots && s->persist == persist) {
+        if (s->emu == emu && s->slots == slots && s->persist == persist && s->alg == alg) {
             match = i;
             break;
         }
@@ -237,7 +238,7 @@ int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float*
 int fa_schedule_count(void) { return schedules().count; }
 
 int fa_schedule_info(int id, int* d, int* emu_every, int* kv_slots, int* persistent,
-                     int* smem_bytes) {
+                     int* algorithm, int* smem_bytes) {
     const ScheduleList& list = schedules();
     if (id < 0 || id >= list.count) return FA_ERR_ARG;
     const fa::Schedule* s = list.items[id];
@@ -245,6 +246,7 @@ int fa_schedule_info(int id, int* d, int* emu_every, int* kv_slots, int* persist
     if (emu_every) *emu_every = s->emu;
     if (kv_slots) *kv_slots = s->slots;
     if (persistent) *persistent = s->persist;
+    if (algorithm) *algorithm = s->alg;
     if (smem_bytes) *smem_bytes = s->smem_bytes;
     return FA_OK;
 }

@@ -1,6 +1,6 @@
 // Compiled schedules of the attention kernel for head dimension 64: the
 // exponential split (EMU) times the K/V ring depth (SLOTS, 16 KiB a slot),
-// plus the two persistent launches for the default exponential split.  First entry
+// plus the two persistent launches and the split-KV ping-pong kernel for the default exponential split.  First entry
 // = default.
 #include "fa_schedules.h"
 
@@ -11,6 +11,8 @@ const Schedule kD64[] = {
     make_schedule<64, 4, 4>(), make_schedule<64, 0, 4>(), make_schedule<64, 2, 4>(),
     make_schedule<64, 4, 8, 1>(), make_schedule<64, 4, 4, 1>(),
     make_schedule<64, 4, 8, 2>(), make_schedule<64, 4, 4, 2>(),
+    make_pp_schedule<64, 4, 8>(), make_pp_schedule<64, 4, 4>(),
+    make_pp_schedule<64, 0, 8>(),
 };
 }  // namespace
 

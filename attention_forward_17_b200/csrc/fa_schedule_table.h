@@ -1,6 +1,6 @@
 // Schedule table of the attention kernel: for each head dimension, masking
 // mode and sequence-length bucket (N <= n_max), the exponential split, the
-// K/V ring depth, the causal launch group and the persistent launch.  Written by
+// K/V ring depth, the causal launch group, the launch form and the algorithm.  Written by
 // attention_forward_17_b200/schedule_search.py on NVIDIA B200 (2026-12-02).
 #pragma once
 
@@ -16,21 +16,22 @@ struct ScheduleTableEntry {
     int slots;
     int group;
     int persist;
+    int alg;
 };
 
 constexpr ScheduleTableEntry kScheduleTable[] = {
-    {128, 0, 2048, 4, 4, 1, 2},
-    {128, 0, 8192, 4, 5, 1, 0},
-    {128, 0, INT64_MAX, 4, 5, 1, 0},
-    {128, 1, 2048, 4, 4, 1, 1},
-    {128, 1, 8192, 4, 5, 16, 0},
-    {128, 1, INT64_MAX, 4, 5, 4, 0},
-    {64, 0, 2048, 4, 8, 1, 2},
-    {64, 0, 8192, 4, 8, 1, 2},
-    {64, 0, INT64_MAX, 4, 8, 1, 0},
-    {64, 1, 2048, 4, 8, 1, 1},
-    {64, 1, 8192, 4, 8, 16, 2},
-    {64, 1, INT64_MAX, 4, 8, 16, 0},
+    {128, 0, 2048, 4, 4, 1, 1, 0},
+    {128, 0, 8192, 4, 5, 1, 1, 0},
+    {128, 0, INT64_MAX, 4, 5, 1, 0, 0},
+    {128, 1, 2048, 4, 4, 1, 1, 0},
+    {128, 1, 8192, 4, 5, 16, 0, 0},
+    {128, 1, INT64_MAX, 4, 5, 2, 0, 0},
+    {64, 0, 2048, 4, 4, 1, 1, 0},
+    {64, 0, 8192, 4, 8, 1, 2, 0},
+    {64, 0, INT64_MAX, 4, 8, 1, 0, 0},
+    {64, 1, 2048, 4, 4, 1, 1, 0},
+    {64, 1, 8192, 4, 8, 16, 2, 0},
+    {64, 1, INT64_MAX, 4, 8, 4, 2, 0},
 };
 
 }  // namespace fa

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include "fa_fwd_kernel.cuh"
+#include "fa_fwd_pp_kernel.cuh"
 
 namespace fa {
 
@@ -21,6 +22,8 @@ struct Schedule {
     int slots;         // K/V ring depth
     int persist;       // launch form: 0 one tile per CTA, 1 persistent (static), 2 persistent by
                        // cluster launch control (tiles taken over from unlaunched CTAs)
+    int alg;           // 0: one softmax pass over every key tile; 1: split-KV ping-pong
+                       // (two softmax groups take alternate key tiles, merged at the end)
     int smem_bytes;    // dynamic shared memory per CTA
     FwdLaunchFn launch[2];   // [causal]
     int (*setup)();          // shared-memory opt-in and register check, both modes
@@ -32,6 +35,45 @@ const Schedule* schedules_d128(int* count);
 const Schedule* schedules_d64(int* count);
 
 // Shared by both definition files.
+template <int D, bool CAUSAL, int EMU, int SLOTS>
+cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const FwdParams& p, unsigned grid, cudaStream_t stream) {
+    fa_fwd_pp_kernel<D, CAUSAL, EMU, SLOTS>
+        <<<grid, kThreads, TileCfg<D, SLOTS>::kSmemBytes, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+template <int D, bool CAUSAL, int EMU, int SLOTS>
+int setup_pp_one() {
+    auto* k = fa_fwd_pp_kernel<D, CAUSAL, EMU, SLOTS>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             TileCfg<D, SLOTS>::kSmemBytes) != cudaSuccess)
+        return -6;
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, k) != cudaSuccess) return -6;
+    if (attr.numRegs * kThreads < kRegSplitTotal) return -6;
+    return 0;
+}
+
+template <int D, int EMU, int SLOTS>
+int setup_pp_both() {
+    const int rc = setup_pp_one<D, false, EMU, SLOTS>();
+    return rc ? rc : setup_pp_one<D, true, EMU, SLOTS>();
+}
+
+template <int D, int EMU, int SLOTS>
+constexpr Schedule make_pp_schedule() {
+    static_assert(TileCfg<D, SLOTS>::kSmemBytes <= 232448, "shared memory per CTA (227 KiB)");
+    return Schedule{D,
+                    EMU,
+                    SLOTS,
+                    0,
+                    1,
+                    TileCfg<D, SLOTS>::kSmemBytes,
+                    {&launch_pp<D, false, EMU, SLOTS>, &launch_pp<D, true, EMU, SLOTS>},
+                    &setup_pp_both<D, EMU, SLOTS>};
+}
+
 template <int D, bool CAUSAL, int EMU, int SLOTS, int PERSIST>
 cudaError_t launch_schedule(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const FwdParams& p, unsigned grid, cudaStream_t stream) {
@@ -70,6 +112,7 @@ constexpr Schedule make_schedule() {
                     EMU,
                     SLOTS,
                     PERSIST,
+                    0,
                     TileCfg<D, SLOTS>::kSmemBytes,
                     {&launch_schedule<D, false, EMU, SLOTS, PERSIST>,
                      &launch_schedule<D, true, EMU, SLOTS, PERSIST>},

@@ -4,7 +4,9 @@ benchmark and validate every candidate, cache the winner).
 
 The search space is what libfa_b200.so has compiled (``schedules()``): the
 share of exponentials evaluated by polynomial on the FMA pipe (none, 1/4, 1/2)
-times the depth of the K/V shared-memory ring, plus two persistent launch
+times the depth of the K/V shared-memory ring, the split-KV ping-pong
+variant of the kernel (two softmax warp groups on alternate key tiles), plus
+two persistent launch
 forms (one CTA per SM walking several query tiles; or one CTA per tile whose
 running CTAs take over the tiles of unlaunched ones by cluster launch
 control), each instantiation already filtered at compile time to fit 227 KiB
@@ -117,7 +119,8 @@ def search(log=print):
                     results.append((s, g, tf, ok))
                     rows.append((d, causal, N, s, g, tf, ok, do, dl))
                     log(f"d={d} causal={int(causal)} N={N:5d} emu={s['emu_every']} "
-                        f"slots={s['kv_slots']} persist={s['persistent']} group={g:2d}  "
+                        f"slots={s['kv_slots']} persist={s['persistent']} alg={s['algorithm']} "
+                        f"group={g:2d}  "
                         f"{tf:7.1f} TFLOP/s  "
                         f"{'ok' if ok else 'REJECTED'} (|dO|={do:.2e}, |dLSE|={dl:.2e})")
                 base = [r for r in results if r[0]["id"] == default["id"] and r[1] == 1][0]
@@ -125,9 +128,10 @@ def search(log=print):
                 if best[2] < base[2] * MARGIN:
                     best = base
                 table.append((d, int(causal), n_max, best[0]["emu_every"], best[0]["kv_slots"], best[1],
-                              best[0]["persistent"]))
+                              best[0]["persistent"], best[0]["algorithm"]))
                 log(f"  -> d={d} causal={int(causal)} N<={n_max or 'max'}: emu={best[0]['emu_every']} "
-                    f"slots={best[0]['kv_slots']} persist={best[0]['persistent']} group={best[1]} "
+                    f"slots={best[0]['kv_slots']} persist={best[0]['persistent']} "
+                    f"alg={best[0]['algorithm']} group={best[1]} "
                     f"({best[2]:.1f} vs default {base[2]:.1f} TFLOP/s)")
                 del q, k, v, o, lse, ref_o, ref_l
                 torch.cuda.empty_cache()
@@ -139,7 +143,7 @@ def write_table(table, device_name, path=TABLE):
     lines = [
         "// Schedule table of the attention kernel: for each head dimension, masking",
         "// mode and sequence-length bucket (N <= n_max), the exponential split, the",
-        "// K/V ring depth, the causal launch group and the persistent launch.  Written by",
+        "// K/V ring depth, the causal launch group, the launch form and the algorithm.  Written by",
         f"// attention_forward_17_b200/schedule_search.py on {device_name} ({stamp}).",
         "#pragma once",
         "",
@@ -155,35 +159,53 @@ def write_table(table, device_name, path=TABLE):
         "    int slots;",
         "    int group;",
         "    int persist;",
+        "    int alg;",
         "};",
         "",
         "constexpr ScheduleTableEntry kScheduleTable[] = {",
     ]
-    for d, causal, n_max, emu, slots, group, persist in table:
+    for d, causal, n_max, emu, slots, group, persist, alg in table:
         nm = "INT64_MAX" if n_max is None else str(n_max)
-        lines.append(f"    {{{d}, {causal}, {nm}, {emu}, {slots}, {group}, {persist}}},")
+        lines.append(f"    {{{d}, {causal}, {nm}, {emu}, {slots}, {group}, {persist}, {alg}}},")
     lines += ["};", "", "}  // namespace fa", ""]
     with open(path, "w") as f:
         f.write("\n".join(lines))
 
 
-def write_report(rows, table, device_name, path):
+def write_report(rows, table, device_name, path, top=5):
+    """Markdown summary: per (d, causal, N) the default schedule and the `top`
+    fastest candidates, then the chosen table."""
     cmd = "python -m attention_forward_17_b200.schedule_search --write --report " + os.path.relpath(path, ROOT)
     out = [f"# Attention schedule search on {device_name}", "",
            "Command (repository root, one GPU):", "", f"    {cmd}", "",
            "B = 16384 / N, H = 16, bf16 N(0,1), seed 0; TFLOP/s by the 4*B*H*N^2*d (non-causal) / half "
            "(causal) convention; per candidate the best of 3 rounds (rotated order) of 3 warm-up + 10 timed "
-           "launches, CUDA events. `ok` = output within the "
-           "parity tolerances of the default schedule's.", "",
-           "| d | causal | N | emu | slots | persistent | group | TFLOP/s | ok |",
-           "|---|---|---|---|---|---|---|---|---|"]
-    for d, causal, N, s, g, tf, ok, _, _ in rows:
-        out.append(f"| {d} | {int(causal)} | {N} | {s['emu_every']} | {s['kv_slots']} | "
-                   f"{s['persistent']} | {g} | {tf:.1f} | {'yes' if ok else 'no'} |")
-    out += ["", "Chosen (table written to `attention_forward_17_b200/csrc/fa_schedule_table.h`):", "",
-            "| d | causal | N <= | emu | slots | group | persistent |", "|---|---|---|---|---|---|---|"]
-    for d, causal, n_max, emu, slots, group, persist in table:
-        out.append(f"| {d} | {causal} | {n_max or 'any'} | {emu} | {slots} | {group} | {persist} |")
+           "launches, CUDA events. `ok` = output within the parity tolerances of the default schedule's. "
+           "launch: 0 one CTA per tile, 1 static persistent, 2 cluster launch control; alg: 0 standard, "
+           "1 split-KV ping-pong. Per problem: the default and the fastest candidates.", ""]
+    keys = []
+    for r in rows:
+        if (r[0], r[1], r[2]) not in keys:
+            keys.append((r[0], r[1], r[2]))
+    for d, causal, N in keys:
+        rs = [r for r in rows if (r[0], r[1], r[2]) == (d, causal, N)]
+        default = rs[0]
+        best = sorted(rs, key=lambda r: -r[5])[:top]
+        out += [f"**d={d} {'causal' if causal else 'non-causal'} N={N}** ({len(rs)} candidates)", "",
+                "| emu | slots | launch | alg | group | TFLOP/s | ok |", "|---|---|---|---|---|---|---|"]
+        for r in [default] + [b for b in best if b is not default]:
+            _, _, _, sch, g, tf, ok, _, _ = r
+            tag = " (default)" if r is default else ""
+            out.append(f"| {sch['emu_every']} | {sch['kv_slots']} | {sch['persistent']} | "
+                       f"{sch['algorithm']} | {g} | {tf:.1f}{tag} | {'yes' if ok else 'no'} |")
+        rejected = [r for r in rs if not r[6]]
+        if rejected:
+            out.append(f"\n{len(rejected)} candidate(s) rejected by the output check.")
+        out.append("")
+    out += ["Chosen (table written to `attention_forward_17_b200/csrc/fa_schedule_table.h`):", "",
+            "| d | causal | N <= | emu | slots | group | launch | alg |", "|---|---|---|---|---|---|---|---|"]
+    for d, causal, n_max, emu, slots, group, persist, alg in table:
+        out.append(f"| {d} | {causal} | {n_max or 'any'} | {emu} | {slots} | {group} | {persist} | {alg} |")
     with open(path, "w") as f:
         f.write("\n".join(out) + "\n")
 

@@ -117,7 +117,11 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
  *                     form (0 = one CTA per query tile, 1 = persistent with a
  *                     static tile assignment, 2 = one CTA per tile whose
  *                     running CTAs take over the tiles of CTAs not launched
- *                     yet, through cluster launch control) and shared memory per CTA of
+ *                     yet, through cluster launch control), algorithm (0 =
+ *                     one softmax pass over every key tile, 1 = split-KV
+ *                     ping-pong: two softmax warp groups take alternate key
+ *                     tiles with their own running statistics and output
+ *                     accumulators, merged per row at the end) and shared memory per CTA of
  *                     schedule `id`; FA_ERR_ARG for an unknown id.  Output
  *                     pointers may be NULL.
  * fa_fwd_pick_schedule - the schedule id and causal group fa_fwd uses for
@@ -133,7 +137,7 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
  */
 int fa_schedule_count(void);
 int fa_schedule_info(int id, int* d, int* emu_every, int* kv_slots, int* persistent,
-                     int* smem_bytes);
+                     int* algorithm, int* smem_bytes);
 int fa_fwd_pick_schedule(int64_t N, int64_t d, int causal, int* schedule_id, int* causal_group);
 int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
                     int64_t H, int64_t N, int64_t d, int causal, float scale, int schedule_id,

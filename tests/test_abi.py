@@ -145,18 +145,19 @@ def test_schedule_registry():
     n = LIB.fa_schedule_count()
     assert n >= 2
     import ctypes
-    vals = [ctypes.c_int() for _ in range(5)]
+    vals = [ctypes.c_int() for _ in range(6)]
     seen = set()
     for i in range(n):
         assert LIB.fa_schedule_info(i, *[ctypes.byref(x) for x in vals]) == fa.FA_OK
-        d, emu, slots, persist, smem = (x.value for x in vals)
+        d, emu, slots, persist, alg, smem = (x.value for x in vals)
         assert d in (64, 128) and emu in (0, 2, 4) and slots >= 4 and persist in (0, 1, 2)
-        assert 0 < smem <= 232448
-        assert (d, emu, slots, persist) not in seen
-        seen.add((d, emu, slots, persist))
+        assert alg in (0, 1) and 0 < smem <= 232448
+        assert (d, emu, slots, persist, alg) not in seen
+        seen.add((d, emu, slots, persist, alg))
     assert any(k[3] == 1 for k in seen) and any(k[3] == 2 for k in seen)
-    assert LIB.fa_schedule_info(n, None, None, None, None, None) == fa.FA_ERR_ARG
-    assert LIB.fa_schedule_info(-1, None, None, None, None, None) == fa.FA_ERR_ARG
+    assert any(k[4] == 1 for k in seen)
+    assert LIB.fa_schedule_info(n, None, None, None, None, None, None) == fa.FA_ERR_ARG
+    assert LIB.fa_schedule_info(-1, None, None, None, None, None, None) == fa.FA_ERR_ARG
     # the first schedule of each head dimension is the default
     assert fa.schedules()[0]["d"] == 128
 

@@ -25,7 +25,7 @@ def run_sched(qt, kt, vt, causal, sid, group):
     return pu.o_f64(o), lse.double().cpu().numpy()
 
 
-@pytest.mark.parametrize("sid", range(24))
+@pytest.mark.parametrize("sid", range(32))
 def test_every_schedule_matches_oracle(cuda_device, sid):
     sched = _schedules()
     if sid >= len(sched):
@@ -44,7 +44,7 @@ def test_causal_groups_cover_every_tile(cuda_device, group):
     (q, k, v), (qt, kt, vt) = pu.inputs(1, 5, 600, 64, seed=group)
     o_ref, lse_ref = oracle.attention_fwd(q, k, v, True, pu.default_scale(64))
     for s in _schedules():
-        if s["d"] == 64 and s["persistent"] != 1:      # the launch forms that use the group
+        if s["d"] == 64 and s["persistent"] != 1 and s["emu_every"] == 4:   # forms that use the group
             o, lse = run_sched(qt, kt, vt, True, s["id"], group)
             pu.check(o, lse, o_ref, lse_ref, f"group {group} schedule {s}")
 
