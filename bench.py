@@ -398,7 +398,8 @@ def run_ours(args, cfg):
         torch.cuda.synchronize()
         barrier()
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
-    launch_ms = {c: statistics.mean(a.elapsed_time(b) for a, b in ev[c]) for c in modes}
+    per_launch = {c: [a.elapsed_time(b) for a, b in ev[c]] for c in modes}
+    launch_ms = {c: statistics.mean(per_launch[c]) for c in modes}
     clocks = clk.summary()
     value = world * f_step * args.steps / (elapsed_ms / 1e3) / 1e12
 
@@ -446,9 +447,34 @@ def run_ours(args, cfg):
                 "algorithmic_bytes_per_launch": 8.0 * B * H * N * d + 4.0 * B * H * N,
                 "per_mode": {("causal" if c else "non_causal"): {
                     "ms_per_launch": launch_ms[c], "tflops": ach[c],
+                    "ms_median": statistics.median(per_launch[c]), "ms_min": min(per_launch[c]),
                     "frac_of_measured_burst": ach[c] / peaks["bf16"],
                     "frac_of_measured_sustained": ach[c] / peaks["bf16_sustained"],
                     "frac_of_datasheet_2250": ach[c] / DATASHEET_BF16_TFLOPS} for c in modes}}
+
+    # ---------------- context: PyTorch scaled-dot-product attention on the same GPU and inputs
+    # (the pages' comparator; library code, timed outside the measured region, never used for parity)
+    context = None
+    if not args.no_context:
+        import torch.nn.functional as F
+        context = {"torch_sdpa_tflops": {}, "note": "torch.nn.functional.scaled_dot_product_attention, "
+                   "bf16, default backend selection, same Q/K/V, 10 launches after 3 warm-ups"}
+        for c in modes:
+            try:
+                run = lambda: F.scaled_dot_product_attention(q, k, v, is_causal=c, scale=1.0 / math.sqrt(d))
+                for _ in range(3):
+                    run()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                a.record(stream)
+                for _ in range(10):
+                    run()
+                b.record(stream)
+                torch.cuda.synchronize()
+                context["torch_sdpa_tflops"]["causal" if c else "non_causal"] = \
+                    flops(B, H, N, d, c) / (a.elapsed_time(b) / 10 / 1e3) / 1e12
+            except Exception as exc:          # a backend may refuse a shape; context only
+                context["torch_sdpa_tflops"]["causal" if c else "non_causal"] = f"unavailable: {exc}"[:120]
 
     # ---------------- CPU baseline (rank 0, N=1 only)
     cpu = None
@@ -473,7 +499,7 @@ def run_ours(args, cfg):
             "pct_of_peak": {"measured_burst": 100 * value / world / peaks["bf16"],
                             "measured_sustained": 100 * value / world / peaks["bf16_sustained"],
                             "datasheet_2250": 100 * value / world / DATASHEET_BF16_TFLOPS},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "context": context,
             "gpu_launches": args.steps * len(modes) * fa.launches_per_call(B, H, N, d),
             "clocks": clocks, "impl": "ours",
         }
@@ -672,6 +698,8 @@ def main():
     ap.add_argument("--causal-group", type=int, default=None,
                     help="pin the causal launch group (default: the search table's choice)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-context", action="store_true",
+                    help="skip the torch SDPA context timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
