@@ -2,48 +2,86 @@
 //
 // Same operation, inputs, outputs and host interface as fa_fwd_kernel (the
 // FlashAttention forward pass of the "TileLang tutorial"); the difference is
-// how the softmax work is spread over the warps.  Each CTA still owns one
-// 128-row query tile, but the key/value tiles are dealt alternately to two
-// softmax groups of four warps:
+// how the softmax work is spread over the warps.  Each CTA owns one 128-row
+// query tile, and the key/value tiles are dealt alternately to two softmax
+// groups of four warps:
 //   group 0 (warps 0-3) takes key tiles 0, 2, 4, ... and group 1 (warps 4-7)
 //   tiles 1, 3, 5, ...; each group keeps its own running maximum and sums for
 //   every row and its own output accumulator O_g in tensor memory.  A thread
 //   owns one whole row (TMEM lane = row, 32x32b access), so row maxima need no
-//   shuffles.  The two groups run one step apart: while one waits for its
-//   scores or works through its exponentials, the other is in a different
-//   phase, and the tensor pipe alternates S = Q K^T and O_g += P V between
-//   them.  At the end the two partial results are merged per row,
+//   shuffles.  At the end the two partial results are merged per row,
 //     M = max(m_0, m_1),  O = (2^(m_0-M) O_0 + 2^(m_1-M) O_1) / (2^(m_0-M) l^_0 + 2^(m_1-M) l^_1),
-//   which is the online-softmax combination of two partial softmaxes.
+//   the online-softmax combination of two partial softmaxes.
+//
+// P goes to shared memory (one 128 x 128 bf16 tile per group, laid out as the
+// 128-byte-swizzled K-major operand the tensor core reads), not over the
+// scores in TMEM.  So a group frees its score buffer as soon as it has read
+// the scores, and the next score product for that group runs while the group
+// is still busy with exponentials; O_g += P V then reads P from shared memory.
+// Before overwriting its P tile (and before rescaling O_g), a group waits
+// until the product two steps back has completed.
 //
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
-// O_1 [256+D, 256+2D).  P_b (bf16 pairs) is written over columns [64,128) of
-// S_b.  Step j uses S_{j&1} and O_{j&1}; S(j) is issued only after the product
-// of step j-2 has completed, so when a group sees its scores its accumulator
-// is already final for the lazy rescale (no extra wait).
+// O_1 [256+D, 256+2D).  Shared memory: Q tile, K/V ring, P_0, P_1, barriers;
+// the per-row statistics exchange of the epilogue reuses the Q tile, which is
+// dead once every product has completed.
 //
-// Roles, barriers, the K/V load sequence, bounded waits and the epilogue
-// conventions are those of fa_fwd_kernel.
+// With P out of TMEM the score issuer no longer waits on a P V product, so it
+// observes only K loads; the ring's parity waits stay sound when a K tile's
+// slot predecessor is always a K tile, i.e. for an even ring depth of at least
+// four (the load sequence alternates V and K after the first three K tiles).
+//
+// Roles, the K/V load sequence, bounded waits and the epilogue conventions are
+// those of fa_fwd_kernel.
 #pragma once
 
 #include "fa_fwd_kernel.cuh"
 
 namespace fa {
 
+template <int D, int SLOTS>
+struct PPCfg {
+    static_assert(SLOTS >= 4 && SLOTS % 2 == 0, "even K/V ring depth of at least four");
+    static constexpr int kTileBytes = kBlockN * D * 2;     // one K or V tile; also the Q tile
+    static constexpr int kBoxes = D / 64;
+    static constexpr int kBoxBytes = 128 * 128;
+    static constexpr int kSlots = SLOTS;
+    static constexpr int kQOff = 0;
+    static constexpr int kSlotOff = kTileBytes;
+    static constexpr int kPOff = kSlotOff + SLOTS * kTileBytes;
+    static constexpr int kPBytes = 128 * 128 * 2;           // one P tile: two 64-key 128B-swizzled boxes
+    static constexpr int kBarOff = kPOff + 2 * kPBytes;
+    static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBarOff + 512;
+    static constexpr uint32_t kTmemCols = 512;
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA (227 KiB)");
+    static_assert(256 + 2 * D <= 512, "two score and two output buffers in TMEM");
+};
+
+template <int kSlots>
+struct alignas(8) PPBarriers {
+    uint64_t kv_full[kSlots];
+    uint64_t kv_empty[kSlots];
+    uint64_t q_full;
+    uint64_t s_full[2];     // S_b computed
+    uint64_t s_free[2];     // the group has read S_b out of TMEM
+    uint64_t p_full[2];     // P_b written to shared memory (and O_b rescaled)
+    uint64_t pv_done[2];    // O_b += P_b V of the latest step on b completed
+    uint64_t o_full;
+    uint32_t tmem_base;
+    volatile uint32_t abort;
+};
+
 template <int D, bool CAUSAL, int EMU, int SLOTS>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using C = TileCfg<D, SLOTS>;
-    static_assert(256 + 2 * D <= 512, "two score and two output buffers in TMEM");
+    using C = PPCfg<D, SLOTS>;
     constexpr uint32_t kColO0 = 256;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_addr);
-    auto* bars = reinterpret_cast<Barriers<C::kSlots>*>(smem + C::kBarOff);
-    // per-row partial statistics of both groups: [group][m | l | l-hat][128]
-    float* red = reinterpret_cast<float*>(smem + C::kRedOff);
+    auto* bars = reinterpret_cast<PPBarriers<C::kSlots>*>(smem + C::kBarOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -57,6 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_kv_empty = smem_u32(&bars->kv_empty[0]);
     const uint32_t bar_q_full = smem_u32(&bars->q_full);
     const uint32_t bar_s_full = smem_u32(&bars->s_full[0]);
+    const uint32_t bar_s_free = smem_u32(&bars->s_free[0]);
     const uint32_t bar_p_full = smem_u32(&bars->p_full[0]);
     const uint32_t bar_pv_done = smem_u32(&bars->pv_done[0]);
     const uint32_t bar_o_full = smem_u32(&bars->o_full);
@@ -70,6 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar_q_full, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_s_full + 8 * b, 1);
+            mbar_init(bar_s_free + 8 * b, 128);
             mbar_init(bar_p_full + 8 * b, 128);
             mbar_init(bar_pv_done + 8 * b, 1);
         }
@@ -100,13 +140,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_w = static_cast<uint32_t>(32 * quarter) << 16;
         const float c = p.scale_log2;
         const uint64_t c2 = f2(c, c);
+        const uint32_t t_s = tmem + lane_w + 128u * g;
         const uint32_t t_o = tmem + lane_w + kColO0 + g * D;
+        // this row of P_g in shared memory: box (keys 64a..), row r, 16-byte
+        // chunk c stored at chunk position c ^ (r % 8) (128-byte swizzle)
+        const uint32_t p_row = base + C::kPOff + g * C::kPBytes + r * 128;
+        const uint32_t sw = static_cast<uint32_t>(r & 7);
 
         float m = -INFINITY;                      // running max of c*s (stale by < 8)
         float l = 0.f, lh = 0.f;                  // sums of the weights, fp32 and bf16-rounded
 
         for (int j = g; j < n_kv; j += 2) {
-            const uint32_t t_s = tmem + lane_w + 128u * g;
             wait_bar(bar_s_full + 8 * g, (j >> 1) & 1, abort, p.status);
             tc_fence_after();
             uint32_t s0[32], s1[32], s2[32], s3[32];
@@ -119,6 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             reg_fence32(s1);
             reg_fence32(s2);
             reg_fence32(s3);
+            // S_g may be overwritten by the next score product from here on
+            tc_fence_before();
+            mbar_arrive(bar_s_free + 8 * g);
 
             const bool masked =
                 (j * kBlockN + kBlockN > p.N) || (CAUSAL && j * kBlockN + kBlockN - 1 > q0);
@@ -132,7 +179,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (96 + i >= lim) s3[i] = __float_as_uint(-INFINITY);
                 }
             }
-            // row maximum, four independent chains
             float x0 = fmaxf(__uint_as_float(s0[0]), __uint_as_float(s0[1]));
             float x1 = fmaxf(__uint_as_float(s1[0]), __uint_as_float(s1[1]));
             float x2 = fmaxf(__uint_as_float(s2[0]), __uint_as_float(s2[1]));
@@ -153,25 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l *= alpha;
                 lh *= alpha;
             }
-            // O_g holds this group's earlier products with the old reference
-            // max; its last product (step j-2) completed before S(j) was issued.
-            if (j >= 2 && __any_sync(0xffffffffu, grow)) {
-#pragma unroll 1
-                for (int q = 0; q < D / 32; ++q) {
-                    uint32_t o[32];
-                    tmem_ld32(t_o + 32 * q, o);
-                    tmem_wait_ld();
-                    reg_fence32(o);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    reg_fence32(o);
-                    tmem_st32(t_o + 32 * q, o);
-                }
-            }
             const float u = (m == -INFINITY) ? 0.f : m;
             const uint64_t negm = f2(-u, -u);
             uint64_t la2 = 0, ha2 = 0;
-            // exponent, exponential, bf16 pair and the two sums for one pair
             const auto pair = [&](uint32_t a, uint32_t b, int pi) -> uint32_t {
                 const uint64_t x2 = fma2(f2(__uint_as_float(a), __uint_as_float(b)), c2, negm);
                 float e0, e1, p0, p1;
@@ -187,8 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ha2 = add2(ha2, f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)));
                 return w;
             };
-            // keys 0..63 -> P words 0..31 (TMEM columns 64..95), keys 64..127 -> words
-            // 32..63 (columns 96..127); every score was read into registers above
+            // word i = keys 2i, 2i+1
             uint32_t pw0[32], pw1[32];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -197,22 +226,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pw1[i] = pair(s2[2 * i], s2[2 * i + 1], 32 + i);
                 pw1[16 + i] = pair(s3[2 * i], s3[2 * i + 1], 48 + i);
             }
-            // registers pinned before the asynchronous TMEM stores (see fa_fwd_kernel)
-            reg_fence32(pw0);
-            reg_fence32(pw1);
-            tmem_st32(t_s + C::kColP, pw0);
-            tmem_st32(t_s + C::kColP + 32, pw1);
             float v0, v1;
             f2_split(la2, v0, v1);
             l += v0 + v1;
             f2_split(ha2, v0, v1);
             lh += v0 + v1;
-            tmem_wait_st();
+
+            if (j >= 2) {
+                // the product of step j-2 has read P_g and is the last update of O_g
+                wait_bar(bar_pv_done + 8 * g, ((j - 2) >> 1) & 1, abort, p.status);
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll 1
+                    for (int q = 0; q < D / 32; ++q) {
+                        uint32_t o[32];
+                        tmem_ld32(t_o + 32 * q, o);
+                        tmem_wait_ld();
+                        reg_fence32(o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        reg_fence32(o);
+                        tmem_st32(t_o + 32 * q, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P row into shared memory: box 0 = words 0..31 (keys 0..63), box 1 = words 32..63
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint32_t off = ((static_cast<uint32_t>(ch) ^ sw) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + off),
+                             "r"(pw0[4 * ch]), "r"(pw0[4 * ch + 1]), "r"(pw0[4 * ch + 2]), "r"(pw0[4 * ch + 3])
+                             : "memory");
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(p_row + C::kBoxBytes + off),
+                             "r"(pw1[4 * ch]), "r"(pw1[4 * ch + 1]), "r"(pw1[4 * ch + 2]), "r"(pw1[4 * ch + 3])
+                             : "memory");
+            }
+            // generic-proxy stores made visible to the tensor core's (async proxy) reads
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
             mbar_arrive(bar_p_full + 8 * g);
         }
 
         // ------------------------------------------------------------ merge + epilogue
+        // every product is done, so Q is dead and its tile holds the statistics exchange
+        wait_bar(bar_o_full, 0, abort, p.status);
+        tc_fence_after();
+        float* red = reinterpret_cast<float*>(smem + C::kQOff);
         red[(g * 3 + 0) * 128 + r] = m;
         red[(g * 3 + 1) * 128 + r] = l;
         red[(g * 3 + 2) * 128 + r] = lh;
@@ -229,8 +289,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float l_t = w0 * l0 + w1 * l1;
         const float inv = lh_t > 0.f ? 1.f / lh_t : 0.f;
         const float s_0 = w0 * inv, s_1 = w1 * inv;
-        wait_bar(bar_o_full, 0, abort, p.status);
-        tc_fence_after();
         const int row = q0 + r;
         const bool valid = row < p.N;
         // this thread writes columns [g*D/2, (g+1)*D/2) of its row
@@ -309,23 +367,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wait_bar(bar_kv_full + 8 * (i % C::kSlots), (i / C::kSlots) & 1, abort, p.status);
                 tc_fence_after();
             };
+            const uint64_t desc_kmaj = smem_desc_sw128(0, 16, 1024);
             if (warp == kMmaWarp) {
                 // ==================================================== score issuer
                 constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false);
-                const uint64_t desc_k = smem_desc_sw128(0, 16, 1024);
-                const uint64_t a0 = desc_k + ((base + C::kQOff) >> 4);
+                const uint64_t a0 = desc_kmaj + ((base + C::kQOff) >> 4);
                 wait_bar(bar_q_full, 0, abort, p.status);
                 tc_fence_after();
                 for (int m = 0; m < n_kv; ++m) {
                     const int b = m & 1;
                     if (m >= 2) {
-                        // S_b still holds P of step m-2 until that product is done
-                        wait_bar(bar_pv_done + 8 * b, ((m - 2) >> 1) & 1, abort, p.status);
+                        // the group has read S_b of step m-2
+                        wait_bar(bar_s_free + 8 * b, ((m - 2) >> 1) & 1, abort, p.status);
                         tc_fence_after();
                     }
                     const int ik = load_index_k(m);
                     wait_kv(ik);
-                    const uint64_t b0 = desc_k + (slot_addr(ik) >> 4);
+                    const uint64_t b0 = desc_kmaj + (slot_addr(ik) >> 4);
                     const uint32_t d_tmem = tmem + 128u * b;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
@@ -335,26 +393,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_commit(bar_s_full + 8 * b);
                     mma_commit(bar_kv_empty + 8 * (ik % C::kSlots));
                 }
-                // every score product has completed before TMEM is released
                 if (n_kv > 0)
                     wait_bar(bar_s_full + 8 * ((n_kv - 1) & 1), ((n_kv - 1) >> 1) & 1, abort, p.status);
             } else {
                 // ==================================================== output issuer
+                // O_b += P_b V: P_b K-major from shared memory (two 64-key boxes,
+                // 16 keys = 32 bytes per MMA), V MN-major as in fa_fwd_kernel
                 constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, true);
                 const uint64_t desc_v = smem_desc_sw128(0, C::kBoxBytes, 1024);
                 for (int t = 0; t < n_kv; ++t) {
                     const int b = t & 1;
                     const int iv = load_index_v(t, n_kv);
-                    // P_t first (it implies every K_m, m <= t, has landed; see TileCfg)
+                    // P_t first (it implies every K_m, m <= t, has landed)
                     wait_bar(bar_p_full + 8 * b, (t >> 1) & 1, abort, p.status);
                     wait_kv(iv);
                     const uint64_t b0 = desc_v + (slot_addr(iv) >> 4);
-                    const uint32_t a_tmem = tmem + 128u * b + C::kColP;
+                    const uint64_t a0 = desc_kmaj + ((base + C::kPOff + b * C::kPBytes) >> 4);
                     const uint32_t d_tmem = tmem + kColO0 + b * D;
 #pragma unroll
-                    for (int kk = 0; kk < kBlockN / 16; ++kk)
-                        mma_ts(d_tmem, a_tmem + kk * 8, b0 + kk * (2048 >> 4), idesc_o,
+                    for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                        const uint32_t a_off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
+                        mma_ss(d_tmem, a0 + a_off, b0 + kk * (2048 >> 4), idesc_o,
                                (t >= 2 || kk > 0) ? 1u : 0u);
+                    }
                     mma_commit(bar_pv_done + 8 * b);
                     mma_commit(bar_kv_empty + 8 * (iv % C::kSlots));
                 }

@@ -2,7 +2,8 @@
 // exponential split (EMU) times the K/V ring depth (SLOTS), every combination
 // that fits 227 KiB of shared memory (a slot is one 32 KiB K or V tile, the Q
 // tile takes another 32 KiB, so at most five slots; at least four keep the
-// ring's parity waits sound), plus the two persistent launches and the split-KV ping-pong kernel (one CTA per SM
+// ring's parity waits sound), plus the two persistent launches and the split-KV ping-pong kernel (P in shared
+// memory, which leaves room for a four-slot ring only) (one CTA per SM
 // walking several query tiles) for the default exponential split.  First
 // entry = default.
 #include "fa_schedules.h"
@@ -14,8 +15,7 @@ const Schedule kD128[] = {
     make_schedule<128, 4, 4>(), make_schedule<128, 0, 4>(), make_schedule<128, 2, 4>(),
     make_schedule<128, 4, 5, 1>(), make_schedule<128, 4, 4, 1>(),
     make_schedule<128, 4, 5, 2>(), make_schedule<128, 4, 4, 2>(),
-    make_pp_schedule<128, 4, 5>(), make_pp_schedule<128, 4, 4>(),
-    make_pp_schedule<128, 0, 5>(),
+    make_pp_schedule<128, 4, 4>(), make_pp_schedule<128, 0, 4>(),
 };
 }  // namespace
 

@@ -20,18 +20,18 @@ struct ScheduleTableEntry {
 };
 
 constexpr ScheduleTableEntry kScheduleTable[] = {
-    {128, 0, 2048, 4, 4, 1, 1, 0},
-    {128, 0, 8192, 4, 5, 1, 1, 0},
-    {128, 0, INT64_MAX, 4, 5, 1, 0, 0},
-    {128, 1, 2048, 4, 4, 1, 1, 0},
-    {128, 1, 8192, 4, 5, 16, 0, 0},
-    {128, 1, INT64_MAX, 4, 5, 2, 0, 0},
-    {64, 0, 2048, 4, 4, 1, 1, 0},
+    {128, 0, 2048, 4, 4, 1, 2, 0},
+    {128, 0, 8192, 4, 5, 1, 0, 0},
+    {128, 0, INT64_MAX, 4, 4, 1, 0, 1},
+    {128, 1, 2048, 4, 4, 16, 2, 0},
+    {128, 1, 8192, 4, 4, 4, 2, 0},
+    {128, 1, INT64_MAX, 4, 4, 16, 0, 1},
+    {64, 0, 2048, 4, 8, 1, 2, 0},
     {64, 0, 8192, 4, 8, 1, 2, 0},
     {64, 0, INT64_MAX, 4, 8, 1, 0, 0},
     {64, 1, 2048, 4, 4, 1, 1, 0},
     {64, 1, 8192, 4, 8, 16, 2, 0},
-    {64, 1, INT64_MAX, 4, 8, 4, 2, 0},
+    {64, 1, INT64_MAX, 4, 8, 16, 0, 1},
 };
 
 }  // namespace fa

@@ -39,7 +39,7 @@ template <int D, bool CAUSAL, int EMU, int SLOTS>
 cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                       const FwdParams& p, unsigned grid, cudaStream_t stream) {
     fa_fwd_pp_kernel<D, CAUSAL, EMU, SLOTS>
-        <<<grid, kThreads, TileCfg<D, SLOTS>::kSmemBytes, stream>>>(tq, tk, tv, p);
+        <<<grid, kThreads, PPCfg<D, SLOTS>::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
@@ -47,7 +47,7 @@ template <int D, bool CAUSAL, int EMU, int SLOTS>
 int setup_pp_one() {
     auto* k = fa_fwd_pp_kernel<D, CAUSAL, EMU, SLOTS>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             TileCfg<D, SLOTS>::kSmemBytes) != cudaSuccess)
+                             PPCfg<D, SLOTS>::kSmemBytes) != cudaSuccess)
         return -6;
     cudaFuncAttributes attr;
     if (cudaFuncGetAttributes(&attr, k) != cudaSuccess) return -6;
@@ -63,13 +63,12 @@ int setup_pp_both() {
 
 template <int D, int EMU, int SLOTS>
 constexpr Schedule make_pp_schedule() {
-    static_assert(TileCfg<D, SLOTS>::kSmemBytes <= 232448, "shared memory per CTA (227 KiB)");
     return Schedule{D,
                     EMU,
                     SLOTS,
                     0,
                     1,
-                    TileCfg<D, SLOTS>::kSmemBytes,
+                    PPCfg<D, SLOTS>::kSmemBytes,
                     {&launch_pp<D, false, EMU, SLOTS>, &launch_pp<D, true, EMU, SLOTS>},
                     &setup_pp_both<D, EMU, SLOTS>};
 }

@@ -19,7 +19,11 @@ times each candidate on a B200 (CUDA events, inputs larger than L2), checks
 its output against the default schedule's (the default is the one the parity
 tests pin to the fp64 oracle; the test suite also runs every schedule against
 the oracle), and writes the fastest into ``csrc/fa_schedule_table.h``.  A
-candidate replaces the default only if it is more than 1 % faster.  Each
+candidate replaces the default only if it is more than 1 % faster.  For the
+longest sequences, which run at the power cap in practice, the default and the
+fastest burst candidates are re-timed under sustained load on wide-range
+scores (q, k ~ N(0, 3^2), the case that exercises the online rescaling) and
+that decides.  Each
 candidate is timed in three rounds that start at different candidates, and its
 best round counts, so power-cap clock drift during the search does not favour
 whichever candidate is timed first.
@@ -44,16 +48,20 @@ BUCKETS = [(1024, 2048), (4096, 8192), (16384, None)]
 GROUPS = [1, 2, 4, 8, 16]
 MARGIN = 1.01
 REPS = 3
+SUSTAINED_FROM_N = 16384   # buckets decided under sustained load
+FINALISTS = 2
+SOAK_S = 0.3
+SUSTAINED_SIGMA = 3.0
 
 
-def _inputs(N, d):
+def _inputs(N, d, sigma_qk=1.0):
     import numpy as np
     import torch
     if ROOT not in sys.path:
         sys.path.insert(0, ROOT)
     import seeded_inputs as si
     B, H = max(1, 16384 // N), 16
-    q, k, v = si.make_qkv(B, H, N, d, seed=0)
+    q, k, v = si.make_qkv(B, H, N, d, seed=0, sigma_qk=sigma_qk)
     dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
     return dev(q), dev(k), dev(v)
 
@@ -72,9 +80,22 @@ def _time(fn, warmup=3, iters=10):
     return a.elapsed_time(b) / iters
 
 
+def _soak(fn, seconds):
+    """Launch fn back to back for about `seconds` (untimed) so the GPU reaches its
+    sustained clock under the power cap."""
+    import time
+    import torch
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        for _ in range(8):
+            fn()
+        torch.cuda.synchronize()
+
+
 def search(log=print):
     import torch
     from . import _binding as fa
+    sustained = []   # (d, causal, N, schedule, group, burst tflops, sustained tflops)
     rows = []        # (d, causal, N, schedule, group, tflops, ok)
     table = []       # (d, causal, n_max, emu, slots, group)
     all_sched = fa.schedules()
@@ -124,9 +145,44 @@ def search(log=print):
                         f"{tf:7.1f} TFLOP/s  "
                         f"{'ok' if ok else 'REJECTED'} (|dO|={do:.2e}, |dLSE|={dl:.2e})")
                 base = [r for r in results if r[0]["id"] == default["id"] and r[1] == 1][0]
-                best = max((r for r in results if r[3]), key=lambda r: r[2])
-                if best[2] < base[2] * MARGIN:
-                    best = base
+                if N >= SUSTAINED_FROM_N:
+                    # long sequences run at the power cap in practice: re-time the default and
+                    # the fastest burst candidates under sustained load and decide on that
+                    # finalists: the default, the fastest burst candidate of every launch form
+                    # and algorithm, and the two fastest overall
+                    ok_rs = sorted((r for r in results if r[3]), key=lambda r: -r[2])
+                    finalists = [base]
+                    classes = {(r[0]["persistent"], r[0]["algorithm"]) for r in ok_rs}
+                    picks = [next(r for r in ok_rs if (r[0]["persistent"], r[0]["algorithm"]) == cl)
+                             for cl in sorted(classes)] + ok_rs[:FINALISTS]
+                    for r in picks:
+                        if all(r is not f for f in finalists):
+                            finalists.append(r)
+                    # decided on the wide score range (q, k ~ N(0, 3^2)), where the online
+                    # rescaling is exercised hardest
+                    q, k, v = _inputs(N, d, SUSTAINED_SIGMA)
+                    sus = [0.0] * len(finalists)
+                    for rep in range(REPS):
+                        start = rep * len(finalists) // REPS
+                        for idx in list(range(start, len(finalists))) + list(range(start)):
+                            s, g, _, _ = finalists[idx]
+                            f = lambda: fa.fa_fwd(q, k, v, causal, out=o, lse=lse, schedule=s["id"],
+                                                  causal_group=g)
+                            _soak(f, SOAK_S)
+                            sus[idx] = max(sus[idx], flop / (_time(f, warmup=0, iters=20) / 1e3) / 1e12)
+                    for (s, g, tf, _), st in zip(finalists, sus):
+                        sustained.append((d, causal, N, s, g, tf, st))
+                        log(f"   sustained: emu={s['emu_every']} slots={s['kv_slots']} "
+                            f"persist={s['persistent']} alg={s['algorithm']} group={g:2d}  {st:7.1f} TFLOP/s")
+                    top = max(range(len(finalists)), key=lambda i: sus[i])
+                    if sus[top] < sus[0] * MARGIN:
+                        top = 0
+                    best = (finalists[top][0], finalists[top][1], sus[top], True)
+                    base = (base[0], base[1], sus[0], True)
+                else:
+                    best = max((r for r in results if r[3]), key=lambda r: r[2])
+                    if best[2] < base[2] * MARGIN:
+                        best = base
                 table.append((d, int(causal), n_max, best[0]["emu_every"], best[0]["kv_slots"], best[1],
                               best[0]["persistent"], best[0]["algorithm"]))
                 log(f"  -> d={d} causal={int(causal)} N<={n_max or 'max'}: emu={best[0]['emu_every']} "
@@ -135,7 +191,7 @@ def search(log=print):
                     f"({best[2]:.1f} vs default {base[2]:.1f} TFLOP/s)")
                 del q, k, v, o, lse, ref_o, ref_l
                 torch.cuda.empty_cache()
-    return rows, table
+    return rows, table, sustained
 
 
 def write_table(table, device_name, path=TABLE):
@@ -172,7 +228,7 @@ def write_table(table, device_name, path=TABLE):
         f.write("\n".join(lines))
 
 
-def write_report(rows, table, device_name, path, top=5):
+def write_report(rows, table, device_name, path, top=5, sustained=()):
     """Markdown summary: per (d, causal, N) the default schedule and the `top`
     fastest candidates, then the chosen table."""
     cmd = "python -m attention_forward_17_b200.schedule_search --write --report " + os.path.relpath(path, ROOT)
@@ -202,6 +258,18 @@ def write_report(rows, table, device_name, path, top=5):
         if rejected:
             out.append(f"\n{len(rejected)} candidate(s) rejected by the output check.")
         out.append("")
+    if sustained:
+        out += [f"Sustained load (N >= {SUSTAINED_FROM_N}: the default, the fastest burst candidate of "
+                f"each launch form and algorithm and the {FINALISTS} fastest overall, on q, k ~ N(0, "
+                f"{SUSTAINED_SIGMA:g}^2) inputs, each launched back to back for {SOAK_S} s before 20 timed "
+                f"launches, best of {REPS} rotated rounds; these decide the bucket; `burst` is the sigma = 1 "
+                f"burst figure):", "",
+                "| d | causal | N | emu | slots | launch | alg | group | burst | sustained |",
+                "|---|---|---|---|---|---|---|---|---|---|"]
+        for d, causal, N, sch, g, tf, st in sustained:
+            out.append(f"| {d} | {int(causal)} | {N} | {sch['emu_every']} | {sch['kv_slots']} | "
+                       f"{sch['persistent']} | {sch['algorithm']} | {g} | {tf:.1f} | {st:.1f} |")
+        out.append("")
     out += ["Chosen (table written to `attention_forward_17_b200/csrc/fa_schedule_table.h`):", "",
             "| d | causal | N <= | emu | slots | group | launch | alg |", "|---|---|---|---|---|---|---|---|"]
     for d, causal, n_max, emu, slots, group, persist, alg in table:
@@ -217,12 +285,12 @@ def main():
     args = ap.parse_args()
     import torch
     name = torch.cuda.get_device_name(0)
-    rows, table = search()
+    rows, table, sustained = search()
     if args.write:
         write_table(table, name)
         print(f"wrote {TABLE}")
     if args.report:
-        write_report(rows, table, name, args.report)
+        write_report(rows, table, name, args.report, sustained=sustained)
         print(f"wrote {args.report}")
 
 

@@ -68,14 +68,16 @@ def load_peaks():
         return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
 
 
-def measured_traffic(workload):
-    """DRAM bytes per non-causal launch from the committed ncu summary, or None
-    when the kernel source changed since the counters were taken (or the
-    summary does not cover this workload)."""
+def measured_traffic(workload, algorithm=0):
+    """DRAM bytes per non-causal launch from the committed ncu summary of the
+    kernel family the headline runs (algorithm 0: fa_fwd_kernel, 1: the split-KV
+    ping-pong kernel), or None when that kernel's source changed since the
+    counters were taken (or the summary does not cover this workload)."""
     if workload != DEFAULT_WORKLOAD:
         return None, None
-    prof = os.path.join(ROOT, "profiles", "fa_fwd_kernel_b1_h64_n4096_d128_ncu.md")
-    src = os.path.join(ROOT, "attention_forward_17_b200", "csrc", "fa_fwd_kernel.cuh")
+    name = "fa_fwd_pp_kernel" if algorithm == 1 else "fa_fwd_kernel"
+    prof = os.path.join(ROOT, "profiles", f"{name}_b1_h64_n4096_d128_ncu.md")
+    src = os.path.join(ROOT, "attention_forward_17_b200", "csrc", f"{name}.cuh")
     try:
         text = open(prof).read()
         want = re.search(r"kernel_source_sha256_16: (\w+)", text).group(1)
@@ -83,8 +85,8 @@ def measured_traffic(workload):
         if want != have:
             return None, "kernel changed since the ncu capture"
         val = float(re.search(r"traffic_bytes_per_launch_noncausal: ([0-9.e+]+)", text).group(1))
-        return val, ("ncu dram__bytes_read+write of one launch at B=1,H=64,N=4096,d=128, scaled x2 by "
-                     "BH*N*d to the workload (profiles/fa_fwd_kernel_b1_h64_n4096_d128_ncu.md)")
+        return val, (f"ncu dram__bytes_read+write of one launch at B=1,H=64,N=4096,d=128, scaled x2 by "
+                     f"BH*N*d to the workload (profiles/{name}_b1_h64_n4096_d128_ncu.md)")
     except (OSError, AttributeError, ValueError):
         return None, None
 
@@ -439,8 +441,11 @@ def run_ours(args, cfg):
     peaks = load_peaks()
     ach = {c: flops(B, H, N, d, c) / (launch_ms[c] / 1e3) / 1e12 for c in modes}
     dominant = max(modes, key=lambda c: launch_ms[c])
-    traffic, traffic_src = measured_traffic(args.workload)
-    roofline = {"bound": "tensor", "kernel": f"fa_fwd_kernel<{d},{str(dominant).lower()}>",
+    sch_dom = schedule_of(N, d, dominant, args.schedule, args.causal_group)
+    traffic, traffic_src = measured_traffic(args.workload, sch_dom["algorithm"])
+    kname = "fa_fwd_pp_kernel" if sch_dom["algorithm"] == 1 else "fa_fwd_kernel"
+    roofline = {"bound": "tensor", "kernel": f"{kname} d={d} {'causal' if dominant else 'non-causal'} "
+                                             f"schedule {sch_dom['id']}",
                 "achieved": ach[dominant], "peak": peaks["bf16"], "unit": "TFLOP/s",
                 "frac": ach[dominant] / peaks["bf16"], "peak_source": peaks["source"] + " burst",
                 "traffic": traffic if dominant is False else None, "traffic_source": traffic_src,
