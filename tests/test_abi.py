@@ -192,3 +192,34 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(bnd, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         bnd._load()
+
+
+def test_schedule_table_entries_are_compiled():
+    # every row of the searched table must name a compiled schedule, or the
+    # dispatch would silently fall back to the first schedule of that head dim
+    import re
+    import os
+    path = os.path.join(os.path.dirname(fa.LIB_PATH), "csrc", "fa_schedule_table.h")
+    rows = re.findall(r"\{(\d+), (\d), (\w+), (\d), (\d), (\d+), (\d), (\d)\},", open(path).read())
+    assert rows, "no table rows parsed"
+    compiled = {(s["d"], s["emu_every"], s["kv_slots"], s["persistent"], s["algorithm"])
+                for s in fa.schedules()}
+    buckets = set()
+    for d, causal, n_max, emu, slots, group, persist, alg in rows:
+        key = (int(d), int(emu), int(slots), int(persist), int(alg))
+        assert key in compiled, f"table row {key} is not a compiled schedule"
+        assert int(group) >= 1
+        buckets.add((int(d), int(causal), n_max))
+    for d in (64, 128):
+        for causal in (0, 1):
+            assert (d, causal, "INT64_MAX") in buckets, f"no open-ended bucket for d={d} causal={causal}"
+    # and the pick for a few sizes agrees with the table row that covers it
+    for d in (64, 128):
+        for causal in (False, True):
+            for N in (1000, 5000, 20000):
+                sid, _ = fa.pick_schedule(N, d, causal)
+                s = fa.schedules()[sid]
+                row = next(r for r in rows if int(r[0]) == d and int(r[1]) == int(causal)
+                           and (r[2] == "INT64_MAX" or N <= int(r[2])))
+                assert (s["emu_every"], s["kv_slots"], s["persistent"], s["algorithm"]) == \
+                    (int(row[3]), int(row[4]), int(row[6]), int(row[7]))

@@ -1,0 +1,121 @@
+"""Model check of the attention kernels' K/V ring protocol, on the CPU.
+
+The producer fills a ring of SLOTS shared-memory slots in a fixed order (per
+query tile: K_0, K_1, K_2, then V_t followed by K_{t+3}); each load's slot is
+reused SLOTS loads later.  A consumer waits for its load with an mbarrier
+*parity* wait, which is only sound if the slot's previous load has already
+completed when the wait starts; otherwise the wait can mistake that older
+phase for its own and read a half-written tile.  So for every load i, the
+consumer of load i must have observed (through its own earlier waits) the
+completion of load i - SLOTS.
+
+What each consumer has observed before it waits, per kernel:
+  score issuer, S(m), one-tile-per-CTA kernel: every K_{m'<m} (it consumed
+      them) and every V_{t<=m-3} (it waited for the product of step m-3);
+  score issuer, S(m), split-KV ping-pong kernel: every K_{m'<m} only (it waits
+      for the softmax to have read S(m-2), not for any product);
+  output issuer, O += P_t V_t (both kernels): every K_{m<=t} (it waited for
+      P_t, which needed S(t), which needed K_t and the K tiles before it) and
+      every V_{t'<t} (it consumed them).
+Persistent launches run several tiles through one ring with global step and
+load counts, so sequences of tiles are checked too (for the launch forms that
+do that; the ping-pong kernel would not be sound across tiles and runs one
+tile per CTA).
+
+This is the reasoning that found a real race (the output issuer used to wait
+for V_t before P_t); the last tests check that the model flags that order and
+a three-slot ring.
+"""
+import random
+
+import pytest
+
+import attention_forward_17_b200 as fa
+
+
+def tile_loads(n):
+    """Load order of one query tile with n key tiles: (kind, key tile index)."""
+    seq = [("K", m) for m in range(min(3, n))]
+    for t in range(n):
+        seq.append(("V", t))
+        if t + 3 < n:
+            seq.append(("K", t + 3))
+    return seq
+
+
+def loads_for(tiles):
+    """Global load sequence over several query tiles; steps counted globally."""
+    seq, base = [], 0
+    for n in tiles:
+        seq += [(k, base + x) for k, x in tile_loads(n)]
+        base += n
+    return seq
+
+
+def observed(kind, step, pred_kind, pred_step, algorithm, v_before_p=False):
+    if kind == "K":                      # score issuer at S(step)
+        if pred_kind == "K":
+            return pred_step < step
+        return algorithm == 0 and pred_step <= step - 3
+    # output issuer at step: after P_step (or, in the faulty order, before it)
+    k_seen = step - 1 if v_before_p else step
+    return (pred_kind == "K" and pred_step <= k_seen) or (pred_kind == "V" and pred_step < step)
+
+
+def violations(tiles, slots, algorithm, v_before_p=False):
+    seq = loads_for(tiles)
+    bad = 0
+    for i, (kind, step) in enumerate(seq):
+        j = i - slots
+        if j >= 0 and not observed(kind, step, *seq[j], algorithm, v_before_p):
+            bad += 1
+    return bad
+
+
+def compiled_rings():
+    return sorted({(s["kv_slots"], s["algorithm"]) for s in fa.schedules()})
+
+
+def compiled_multi_tile_rings():
+    """Rings that continue across query tiles (the persistent launch forms)."""
+    return sorted({(s["kv_slots"], s["algorithm"]) for s in fa.schedules() if s["persistent"]})
+
+
+@pytest.mark.parametrize("slots,algorithm", compiled_rings())
+def test_every_compiled_ring_is_sound_for_one_tile(slots, algorithm):
+    for n in range(1, 70):
+        assert violations([n], slots, algorithm) == 0, f"n={n}"
+
+
+@pytest.mark.parametrize("slots,algorithm", compiled_multi_tile_rings())
+def test_every_compiled_ring_is_sound_across_tiles(slots, algorithm):
+    rng = random.Random(slots * 10 + algorithm)
+    for _ in range(2000):
+        tiles = [rng.randint(1, 20) for _ in range(rng.randint(1, 6))]
+        assert violations(tiles, slots, algorithm) == 0, f"tiles={tiles}"
+
+
+def test_model_flags_the_old_wait_order():
+    # waiting for V_t before P_t was racy at the old default depth of five
+    assert sum(violations([n], 5, 0, v_before_p=True) for n in range(1, 40)) > 0
+
+
+def test_model_flags_a_three_slot_ring():
+    assert sum(violations([n], 3, 0) for n in range(1, 40)) > 0
+    assert sum(violations([n], 3, 1) for n in range(1, 40)) > 0
+
+
+def test_ping_pong_kernel_is_never_persistent():
+    # across a tile boundary the ping-pong score issuer could reach a K tile whose
+    # slot predecessor is a V tile of the previous query tile, which it never
+    # observes: the model flags it, so that kernel runs one tile per CTA only
+    rng = random.Random(7)
+    assert any(violations([rng.randint(1, 20) for _ in range(4)], 4, 1) for _ in range(200))
+    assert not any(s["persistent"] for s in fa.schedules() if s["algorithm"] == 1)
+
+
+def test_model_flags_an_odd_ring_for_the_ping_pong_kernel():
+    # with P in shared memory the score issuer observes no V load, so a K tile's
+    # slot predecessor must itself be a K tile: odd depths break that
+    assert sum(violations([n], 5, 1) for n in range(1, 40)) > 0
+    assert all(s["kv_slots"] % 2 == 0 for s in fa.schedules() if s["algorithm"] == 1)
