@@ -684,14 +684,50 @@ def bench_vector_add(args):
     print(json.dumps(line), flush=True)
 
 
+def bench_sweep(args):
+    """Sequence-length sweep: N in 512..32768 with B = max(1, 16384/N), H = 16,
+    d in {64, 128}, bf16 N(0,1), both masks; one JSON line per point with the
+    TFLOP/s of each mask (mean of `--steps` launches after `--warmup`, short
+    back-to-back bursts) and the fraction of the measured bf16 burst peak."""
+    import numpy as np
+    import torch
+    import attention_forward_17_b200 as fa
+    import seeded_inputs as si
+    peaks = load_peaks()
+    for d in (64, 128):
+        for N in (512, 1024, 2048, 4096, 8192, 16384, 32768):
+            B, H = max(1, 16384 // N), 16
+            bits = si.make_qkv(B, H, N, d, seed=0)
+            q, k, v = (torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).cuda() for b in bits)
+            o = torch.empty_like(q)
+            lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+            res = {}
+            for c in (False, True):
+                run = lambda: fa.fa_fwd(q, k, v, causal=c, out=o, lse=lse)
+                for _ in range(args.warmup):
+                    run()
+                ms, _ = _event_loop(run, args.steps)
+                tf = flops(B, H, N, d, c) / (ms / 1e3) / 1e12
+                res["causal" if c else "non_causal"] = {
+                    "ms_per_launch": ms, "tflops": tf, "frac_of_measured_burst": tf / peaks["bf16"],
+                    "schedule": schedule_of(N, d, c)}
+            print(json.dumps({"suite": "sweep", "metric": METRIC, "unit": "TFLOP/s", "B": B, "H": H,
+                              "N": N, "d": d, "dtype": "bf16", "data": "synthetic N(0,1), seed 0",
+                              "steps": args.steps, "warmup": args.warmup, "modes": res,
+                              "peak": peaks["bf16"], "impl": "ours"}), flush=True)
+            del q, k, v, o, lse
+            torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--suite", choices=["attention", "next"], default="attention",
-                    help="'next' measures the kernels beyond the attention path, one line each")
+    ap.add_argument("--suite", choices=["attention", "next", "sweep"], default="attention",
+                    help="'next' measures the kernels beyond the attention path, one line each; "
+                         "'sweep' the sequence-length sweep, one line per (d, N)")
     ap.add_argument("--next", nargs="+", choices=["row_softmax", "gemm", "vector_add"],
                     default=["row_softmax", "gemm", "vector_add"],
                     help="kernels measured by --suite next")
@@ -714,6 +750,9 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     cfg = WORKLOADS[args.workload]
+    if args.suite == "sweep":
+        bench_sweep(args)
+        return
     if args.suite == "next":
         for name in args.next:
             {"row_softmax": bench_row_softmax, "gemm": bench_gemm,
