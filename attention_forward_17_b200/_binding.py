@@ -44,7 +44,7 @@ class FaError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is not built; run `python -m attention_forward_17_b200.build` "
+            f"{LIB_PATH} is not built; run `python attention_forward_17_b200/build.py` "
             "(there is no non-CUDA fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     lib.fa_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.c_int,

@@ -223,3 +223,18 @@ def test_schedule_table_entries_are_compiled():
                            and (r[2] == "INT64_MAX" or N <= int(r[2])))
                 assert (s["emu_every"], s["kv_slots"], s["persistent"], s["algorithm"]) == \
                     (int(row[3]), int(row[4]), int(row[6]), int(row[7]))
+
+
+def test_build_entry_does_not_need_the_library():
+    # the build step must not import the package (its __init__ loads the library
+    # the build step is about to create), so a fresh checkout can build
+    import subprocess
+    import sys
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys, __graft_entry__ as g\n"
+            "m = g._load_by_path('_b', 'attention_forward_17_b200/build.py')\n"
+            "assert callable(m.build) and m.library_path().endswith('libfa_b200.so')\n"
+            "assert 'attention_forward_17_b200' not in sys.modules, 'package imported'\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
