@@ -74,9 +74,11 @@ typedef enum {
  *
  * o and lse must not overlap q, k or v (not checked).  Should a device-side
  * pipeline wait ever exceed about two seconds (it cannot in correct
- * operation), the affected query rows receive LSE = NaN and the kernel still
- * terminates; use fa_fwd_status to also receive FA_ERR_TIMEOUT in a status
- * word.
+ * operation), the CTA involved gives up: the rows of the query tile it is on
+ * receive LSE = NaN, tiles a persistent CTA had not reached yet are left
+ * unwritten, and the kernel still terminates (in-flight copies and products
+ * are drained first).  The outputs are then undefined; use fa_fwd_status to
+ * receive FA_ERR_TIMEOUT in a status word, the reliable signal.
  */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
            int64_t N, int64_t d, int causal, float scale, void* stream);
