@@ -10,7 +10,10 @@ seeded input generator in ``seeded_inputs``.
   P = row softmax of S,  O = P V,  LSE_i = ln sum_j exp(S[i, j])
 as in the FlashAttention section of the TileLang tutorial (fused forward over
 Q/K/V tiles, validated against scaled-dot-product attention, causal and
-non-causal).  ``row_softmax`` is the tutorial's row-wise softmax, ``gemm`` its
+non-causal).  ``attention_fwd_strips`` computes the same definition with
+fp64 library matrix products (torch on the CPU) as its steps, a strip of
+complete query rows at a time, so whole outputs of the large workloads finish
+in seconds; it is pinned against ``attention_fwd``.  ``row_softmax`` is the tutorial's row-wise softmax, ``gemm`` its
 tiled matrix multiplication with the optional fused bias / bias + GELU
 epilogue, ``vector_add`` its elementwise addition.  Every function here is
 pinned by ``tests/test_oracle.py`` or ``tests/test_oracle_gemm.py``.
@@ -96,6 +99,52 @@ def attention_rows(q, k, v, causal: bool, scale: float, rows, threads: int = 0):
                                       o.ctypes.data, lse.ctypes.data, int(threads))
     if rc != 0:
         raise RuntimeError(f"oracle_attention_rows failed ({rc})")
+    return o, lse
+
+
+def attention_fwd_strips(q, k, v, causal: bool, scale: float, strip: int = 1024):
+    """The definition of ``attention_fwd`` with fp64 matrix products as steps.
+
+    For each (b, h) and each strip of up to ``strip`` complete query rows
+    [r0, r1):
+      S = scale * Q[r0:r1] K^T              (fp64 matrix product; under the causal
+                                             mask only keys j < r1 can be visible)
+      S[i, j] = -inf where j > i (causal)
+      m = max_j S,  E = exp(S - m),  l = sum_j E
+      O = (E V) / l,  LSE = m + ln l
+    Every row sees its complete score row, as in ``attention_fwd``; only the
+    summation order inside the products differs (a library fp64 product).
+    Returns fp64 O [B,H,N,d] and LSE [B,H,N].  Rows whose keys are all masked
+    cannot occur with the top-left mask and equal lengths.
+    """
+    import torch
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    B, H, N, d = q.shape
+    assert k.shape == q.shape and v.shape == q.shape
+
+    def widen(b):
+        # bf16 bits -> fp32 (exact: the bits are the upper half of the fp32) -> fp64
+        u = torch.from_numpy(b.astype(np.int32) << 16)
+        return u.view(torch.float32).to(torch.float64)
+
+    o = np.zeros((B, H, N, d), dtype=np.float64)
+    lse = np.zeros((B, H, N), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            qh, kh, vh = widen(q[b, h]), widen(k[b, h]), widen(v[b, h])
+            for r0 in range(0, N, strip):
+                r1 = min(N, r0 + strip)
+                nk = r1 if causal else N
+                s = scale * (qh[r0:r1] @ kh[:nk].T)
+                if causal:
+                    i = torch.arange(r0, r1).unsqueeze(1)
+                    j = torch.arange(nk).unsqueeze(0)
+                    s.masked_fill_(j > i, float("-inf"))
+                m = s.max(dim=1, keepdim=True).values
+                e = torch.exp(s - m)
+                l = e.sum(dim=1, keepdim=True)
+                o[b, h, r0:r1] = ((e @ vh[:nk]) / l).numpy()
+                lse[b, h, r0:r1] = (m + torch.log(l)).squeeze(1).numpy()
     return o, lse
 
 

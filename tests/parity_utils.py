@@ -2,7 +2,9 @@
 kernel call, and the tolerance check against the fp64 oracle."""
 from __future__ import annotations
 
+import json
 import math
+import os
 
 import numpy as np
 
@@ -53,6 +55,10 @@ def check(o_gpu: np.ndarray, lse_gpu: np.ndarray, o_ref: np.ndarray, lse_ref: np
     rel_l2 = float(np.linalg.norm(o_gpu - o_ref) / denom) if denom > 0 else float(np.linalg.norm(o_gpu))
     lse_err = float(np.abs(lse_gpu[fin] - lse_ref[fin]).max()) if fin.any() else 0.0
     m = dict(o_max_abs=max_abs, o_rel_l2=rel_l2, lse_max_abs=lse_err)
+    log = os.environ.get("FA_PARITY_LOG")
+    if log:     # one JSON line per comparison, for the record of a GPU run
+        with open(log, "a") as f:
+            f.write(json.dumps(dict(what=what, rows=int(o_ref.size // max(1, o_ref.shape[-1])), **m)) + "\n")
     assert max_abs <= O_MAX_ABS, f"{what}: O max-abs {max_abs:.3e} > {O_MAX_ABS} ({m})"
     assert rel_l2 <= O_REL_L2, f"{what}: O rel-L2 {rel_l2:.3e} > {O_REL_L2} ({m})"
     assert lse_err <= LSE_MAX_ABS, f"{what}: LSE max-abs {lse_err:.3e} > {LSE_MAX_ABS} ({m})"

@@ -207,6 +207,52 @@ def test_rows_entry_matches_full():
         np.testing.assert_array_equal(rl, lse.reshape(-1)[rows])
 
 
+# ---------------------------------------------------------------- strip form (fp64 matrix products)
+@pytest.mark.parametrize("N,strip", [(130, 64), (700, 256), (257, 1024), (1, 16)])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("sigma", [1.0, 3.0])
+def test_strips_match_plain_loops(N, strip, causal, sigma):
+    # the strip form against the per-row loops: strip edges inside and past N,
+    # wide and narrow score ranges, both masks
+    q, k, v = rand_qkv(2, 2, N, 64, seed=N + strip, sigma=sigma)
+    o, lse = oracle.attention_fwd(q, k, v, causal, 0.125)
+    so, sl = oracle.attention_fwd_strips(q, k, v, causal, 0.125, strip=strip)
+    np.testing.assert_allclose(so, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(sl, lse, rtol=1e-13, atol=1e-12)
+
+
+def test_strips_worked_examples():
+    cases = json.load(open(GOLDEN))["cases"]
+    env = {"e": math.e, "log": math.log}
+    for c in cases:
+        q = bits(np.array(c["q"])[None, None])
+        k = bits(np.array(c["k"])[None, None])
+        v = bits(np.array(c["v"])[None, None])
+        o, lse = oracle.attention_fwd_strips(q, k, v, c["causal"], c["scale"], strip=2)
+        exp_o = np.array([[eval(x, env) for x in row] for row in c["O"]])
+        exp_l = np.array([eval(x, env) for x in c["LSE"]])
+        np.testing.assert_allclose(o[0, 0], exp_o, rtol=0, atol=1e-13, err_msg=c["name"])
+        np.testing.assert_allclose(lse[0, 0], exp_l, rtol=0, atol=1e-13, err_msg=c["name"])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_strips_zero_q_prefix_means(causal):
+    # Q = 0: uniform weights over the visible keys (closed form, strips of 100 rows)
+    N, d = 333, 8
+    q, k, v = rand_qkv(1, 1, N, d, seed=21)
+    q = np.zeros_like(q)
+    o, lse = oracle.attention_fwd_strips(q, k, v, causal, 0.5, strip=100)
+    vf = f64(v)[0, 0]
+    if causal:
+        ref = np.cumsum(vf, 0) / np.arange(1, N + 1)[:, None]
+        ref_l = np.log(np.arange(1, N + 1))
+    else:
+        ref = np.broadcast_to(vf.mean(0), (N, d))
+        ref_l = np.full(N, math.log(N))
+    np.testing.assert_allclose(o[0, 0], ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse[0, 0], ref_l, rtol=0, atol=1e-12)
+
+
 def test_thread_count_does_not_change_result():
     q, k, v = rand_qkv(1, 2, 200, 64, seed=11)
     a = oracle.attention_fwd(q, k, v, False, 0.125, threads=1)

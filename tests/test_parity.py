@@ -75,14 +75,34 @@ def sampled_case(B, H, N, d, causal, sigma=1.0, count=192, seed=0):
     return m
 
 
-def test_b2_h16_n4096_d128_causal(cuda_device):
-    sampled_case(2, 16, 4096, 128, True)
+# --------------------------------------------------------------- full sizes, every element
+def whole_case(B, H, N, d, causal, sigma=1.0, seed=0):
+    """Every element of O and LSE at a full workload size against the strip
+    form of the oracle (fp64 matrix products), rel-L2 over the whole tensor."""
+    (q, k, v), (qt, kt, vt) = pu.inputs(B, H, N, d, seed=seed, sigma_qk=sigma)
+    scale = pu.default_scale(d)
+    o, lse = pu.run(qt, kt, vt, causal)
+    o_g, l_g = pu.o_f64(o), lse.cpu().numpy().astype(np.float64)
+    del o, lse, qt, kt, vt
+    o_ref, lse_ref = oracle.attention_fwd_strips(q, k, v, causal, scale)
+    m = pu.check(o_g, l_g, o_ref, lse_ref,
+                 f"whole B{B} H{H} N{N} d{d} causal={causal} sigma={sigma:.4g}")
+    print(f"whole-output parity B={B} H={H} N={N} d={d} causal={causal} sigma={sigma:.4g}: {m}")
+    return m
+
+
+def test_b2_h16_n4096_d128_causal_whole(cuda_device):
+    whole_case(2, 16, 4096, 128, True)
 
 
 @pytest.mark.parametrize("sigma", [3.0, 3.0 ** 0.5])
 @pytest.mark.parametrize("causal", [False, True])
-def test_b1_h32_n16384_d128_wide(cuda_device, sigma, causal):
-    sampled_case(1, 32, 16384, 128, causal, sigma=sigma)
+def test_b1_h32_n16384_d128_wide_whole(cuda_device, sigma, causal):
+    whole_case(1, 32, 16384, 128, causal, sigma=sigma)
+
+
+def test_b2_h16_n4096_d128_causal(cuda_device):
+    sampled_case(2, 16, 4096, 128, True)
 
 
 @pytest.mark.parametrize("N", [512, 1024, 2048, 4096, 8192, 16384, 32768])
