@@ -65,6 +65,9 @@ def _load():
     lib.fa_fwd_schedule.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.c_int,
                                     ctypes.c_float, ctypes.c_int, ctypes.c_int, _vp, _vp]
     lib.fa_fwd_schedule.restype = ctypes.c_int
+    lib.fa_fwd_rescale_stats.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64,
+                                         ctypes.c_int, ctypes.c_float, ctypes.c_int, _vp, _vp]
+    lib.fa_fwd_rescale_stats.restype = ctypes.c_int
     lib.fa_schedule_count.argtypes = []
     lib.fa_schedule_count.restype = ctypes.c_int
     lib.fa_schedule_info.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp]
@@ -194,6 +197,37 @@ def fa_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, 
     if rc != FA_OK:
         raise FaError(rc)
     return out, lse
+
+
+def rescale_stats(q, k, v, causal: bool = False, scale: float | None = None,
+                  schedule: int | None = None):
+    """Runs the forward pass once with the rescale counters on; returns
+    (O, LSE, warp_steps_rescaled, row_steps_rescaled, warp_steps_total): how many
+    (warp, key tile) steps and (row, key tile) steps rescaled the output
+    accumulator, and the number of (warp, key tile) steps the two-query-tile
+    kernel executed.  Only that kernel counts (other schedules report zeros)."""
+    import torch
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    counts = torch.zeros(2, dtype=torch.int64, device=q.device)
+    s = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        rc = lib.fa_fwd_rescale_stats(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                      lse.data_ptr(), B, H, N, d, int(bool(causal)), float(scale),
+                                      -1 if schedule is None else int(schedule),
+                                      counts.data_ptr(), s)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_rescale_stats")
+    torch.cuda.synchronize(q.device)
+    # (warp, key tile) steps of the two-query-tile kernel: 4 warps per query tile,
+    # key tiles up to the diagonal under the mask
+    nq, nk = (N + 127) // 128, (N + 127) // 128
+    steps = sum(min(nk, t + 1) if causal else nk for t in range(nq))
+    return out, lse, int(counts[0].item()), int(counts[1].item()), 4 * B * H * steps
 
 
 def fa_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal: bool = False,

@@ -49,6 +49,33 @@ DeviceState g_devices[kMaxDevices];
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// The copy streams and events of fa_fwd_host's pipelined path, one set per
+// device, created on first use and kept for the life of the process.
+constexpr int kHostChunks = 8;
+struct HostPipe {
+    std::mutex mu;
+    std::once_flag once;
+    int status = FA_OK;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[2 * kHostChunks + 2] = {};
+};
+HostPipe g_pipes[kMaxDevices];
+
+int host_pipe(HostPipe** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+    HostPipe& hp = g_pipes[dev];
+    std::call_once(hp.once, [&] {
+        bool ok = cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking) == cudaSuccess;
+        for (int i = 0; ok && i < 2 * kHostChunks + 2; ++i)
+            ok = cudaEventCreateWithFlags(&hp.ev[i], cudaEventDisableTiming) == cudaSuccess;
+        hp.status = ok ? FA_OK : FA_ERR_CUDA;
+    });
+    *out = &hp;
+    return hp.status;
+}
+
 // Every compiled schedule, head dimension 128 first, then 64.  Ids are
 // positions in this list.
 struct ScheduleList {
@@ -168,7 +195,7 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
 // schedule_id < 0 and group < 1 take the table's choice.
 int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
             int64_t N, int64_t d, int causal, float scale, int schedule_id, int group,
-            int* dev_status, void* stream) {
+            int* dev_status, void* stream, unsigned long long* rescale_stats = nullptr) {
     int rc = check_args(q, k, v, o, lse, B, H, N, d, scale);
     if (rc == 1) return FA_OK;
     if (rc != 0) return rc;
@@ -183,9 +210,9 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
     if ((rc = current_device_ready(&sms)) != FA_OK) return rc;
     if ((rc = encoder_ready()) != FA_OK) return rc;
     const int64_t BH = B * H;
-    alignas(64) CUtensorMap tq, tk, tv;
+    alignas(64) CUtensorMap tq, tk, tv, to;
     if (encode_qkv_map(&tq, q, BH, N, d) || encode_qkv_map(&tk, k, BH, N, d) ||
-        encode_qkv_map(&tv, v, BH, N, d))
+        encode_qkv_map(&tv, v, BH, N, d) || encode_qkv_map(&to, o, BH, N, d))
         return FA_ERR_CUDA;
     fa::FwdParams p;
     p.o = static_cast<__nv_bfloat16*>(o);
@@ -196,15 +223,19 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
     p.n_qtile = static_cast<int>((N + fa::kBlockM - 1) / fa::kBlockM);
     p.group = static_cast<int>(group < BH ? group : BH);
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.rescale_stats = rescale_stats;
     int64_t grid = BH * p.n_qtile;
     if (grid > 0x7fffffffLL) return FA_ERR_SHAPE;
     const fa::Schedule* sch = list.items[schedule_id];
-    if (sch->persist == 1) {
+    if (sch->alg == 2) {
+        // two query tiles per CTA
+        grid = BH * ((p.n_qtile + 1) / 2);
+    } else if (sch->persist == 1) {
         // one CTA per SM; causal work comes in units of two query tiles
         const int64_t units = causal ? BH * ((p.n_qtile + 1) / 2) : grid;
         grid = units < sms ? units : sms;
     }
-    const cudaError_t e = sch->launch[causal ? 1 : 0](tq, tk, tv, p, static_cast<unsigned>(grid),
+    const cudaError_t e = sch->launch[causal ? 1 : 0](tq, tk, tv, to, p, static_cast<unsigned>(grid),
                                                        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -233,6 +264,18 @@ int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float*
     }
     return run_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, schedule_id, causal_group,
                    dev_status, stream);
+}
+
+int fa_fwd_rescale_stats(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+                         int schedule_id, unsigned long long* dev_counts, void* stream) {
+    const int rc = check_args(q, k, v, o, lse, B, H, N, d, scale);
+    if (rc == 1) return FA_OK;
+    if (rc != 0) return rc;
+    if (!dev_counts) return FA_ERR_NULL;
+    if (schedule_id < -1) return FA_ERR_ARG;
+    return run_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, schedule_id, 0, nullptr, stream,
+                   dev_counts);
 }
 
 int fa_schedule_count(void) { return schedules().count; }
@@ -272,13 +315,13 @@ int fa_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, fl
     const int64_t BH = B * H;
     const size_t slice = static_cast<size_t>(N * d);      // elements of one (b, h) slice
     // Chunks of (b, h) slices, each large enough for about four waves of
-    // query tiles, at most eight: chunk c uploads while chunk c-1 computes and
-    // chunk c-2 downloads.
+    // query tiles, at most kHostChunks: chunk c uploads while chunk c-1
+    // computes and chunk c-2 downloads.
     const int64_t n_qtile = (N + fa::kBlockM - 1) / fa::kBlockM;
     int64_t per = (4 * static_cast<int64_t>(sms) + n_qtile - 1) / n_qtile;
     if (per < 1) per = 1;
     int64_t chunks = (BH + per - 1) / per;
-    if (chunks > 8) chunks = 8;
+    if (chunks > kHostChunks) chunks = kHostChunks;
     per = (BH + chunks - 1) / chunks;
     chunks = (BH + per - 1) / per;
     auto h2d = [&](int64_t c0, int64_t n, cudaStream_t st) {
@@ -305,41 +348,43 @@ int fa_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, fl
     };
     if (chunks <= 1) {
         if (!h2d(0, BH, s)) return FA_ERR_CUDA;
-        if ((rc = run_chunk(0, BH)) != FA_OK) return rc;
+        if (run_chunk(0, BH) != FA_OK) return FA_ERR_CUDA;
         return d2h(0, BH, s) ? FA_OK : FA_ERR_CUDA;
     }
-    // Copies run on two streams of their own, ordered against `stream` by
-    // events; `stream` waits for the last download, so its completion still
-    // means the whole call is done.  Streams and events are released by the
-    // runtime once their work has completed.
-    cudaStream_t s_in = nullptr, s_out = nullptr;
-    cudaEvent_t ev[2 * 8 + 2] = {};
-    const int n_ev = static_cast<int>(2 * chunks + 2);
-    bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess;
-    for (int i = 0; ok && i < n_ev; ++i)
-        ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+    // Copies run on the device's two library-owned copy streams, ordered
+    // against `stream` by events; `stream` waits for the last download, so its
+    // completion means the whole call is done.  The streams and events are
+    // created on the first pipelined call on a device and kept; the lock makes
+    // concurrent calls take turns enqueueing (it is never held while waiting
+    // for the GPU).
+    HostPipe* pipe = nullptr;
+    if ((rc = host_pipe(&pipe)) != FA_OK) return rc;
+    std::lock_guard<std::mutex> lock(pipe->mu);
+    cudaEvent_t* ev = pipe->ev;
     cudaEvent_t ev_start = ev[0], ev_done = ev[1];
-    ok = ok && cudaEventRecord(ev_start, s) == cudaSuccess &&
-         cudaStreamWaitEvent(s_in, ev_start, 0) == cudaSuccess &&
-         cudaStreamWaitEvent(s_out, ev_start, 0) == cudaSuccess;
+    bool ok = cudaEventRecord(ev_start, s) == cudaSuccess &&
+              cudaStreamWaitEvent(pipe->s_in, ev_start, 0) == cudaSuccess &&
+              cudaStreamWaitEvent(pipe->s_out, ev_start, 0) == cudaSuccess;
     for (int64_t c = 0; ok && c < chunks; ++c) {
         const int64_t c0 = c * per, n = (c0 + per <= BH) ? per : BH - c0;
         cudaEvent_t ev_in = ev[2 + 2 * c], ev_k = ev[3 + 2 * c];
-        ok = h2d(c0, n, s_in) && cudaEventRecord(ev_in, s_in) == cudaSuccess &&
+        ok = h2d(c0, n, pipe->s_in) && cudaEventRecord(ev_in, pipe->s_in) == cudaSuccess &&
              cudaStreamWaitEvent(s, ev_in, 0) == cudaSuccess;
-        if (ok && (rc = run_chunk(c0, n)) != FA_OK) break;
+        ok = ok && run_chunk(c0, n) == FA_OK;
         ok = ok && cudaEventRecord(ev_k, s) == cudaSuccess &&
-             cudaStreamWaitEvent(s_out, ev_k, 0) == cudaSuccess && d2h(c0, n, s_out);
+             cudaStreamWaitEvent(pipe->s_out, ev_k, 0) == cudaSuccess && d2h(c0, n, pipe->s_out);
     }
-    ok = ok && rc == FA_OK && cudaEventRecord(ev_done, s_out) == cudaSuccess &&
-         cudaStreamWaitEvent(s, ev_done, 0) == cudaSuccess;
-    for (int i = 0; i < n_ev; ++i)
-        if (ev[i]) cudaEventDestroy(ev[i]);
-    if (s_in) cudaStreamDestroy(s_in);
-    if (s_out) cudaStreamDestroy(s_out);
-    if (rc != FA_OK) return rc;
-    return ok ? FA_OK : FA_ERR_CUDA;
+    if (ok) {
+        ok = cudaEventRecord(ev_done, pipe->s_out) == cudaSuccess &&
+             cudaStreamWaitEvent(s, ev_done, 0) == cudaSuccess;
+        if (ok) return FA_OK;
+    }
+    // Something failed after work was enqueued: make `stream` wait for every
+    // copy already queued on the copy streams (their host buffers must stay
+    // valid until then), then report the failure.
+    for (cudaStream_t cs : {pipe->s_in, pipe->s_out})
+        if (cudaEventRecord(ev_done, cs) == cudaSuccess) cudaStreamWaitEvent(s, ev_done, 0);
+    return FA_ERR_CUDA;
 }
 
 int fa_selftest_wait_timeout(int* dev_status, int64_t limit_us, int arrive, void* stream) {

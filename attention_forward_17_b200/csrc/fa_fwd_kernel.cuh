@@ -69,16 +69,6 @@ constexpr uint64_t kWaitLimitAbortNs = 1000000ull;    // 1 ms once the CTA has a
 constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kRegsOther = 88;
 constexpr int kRegSplitTotal = 2 * 128 * kRegsSoftmax + 128 * kRegsOther;  // 64512 = 384 x 168
-// Sum the bf16-rounded weights with mixed-precision adds that read the 16-bit
-// halves directly (1) or by widening the halves to fp32 first (0).
-#ifndef FA_LHAT_MIXED_ADD
-#define FA_LHAT_MIXED_ADD 0
-#endif
-// Evaluate the exponentials of a tile in separate passes (all exponents, then
-// all exponentials in place, then packing and sums) instead of pair by pair.
-#ifndef FA_SOFTMAX_PHASED
-#define FA_SOFTMAX_PHASED 1
-#endif
 
 // Schedule knobs (template parameters of the kernel, chosen per problem by
 // the host from a table the schedule search writes):
@@ -138,6 +128,9 @@ struct FwdParams {
     int n_qtile;             // ceil(N / 128)
     int group;               // causal launch order: heads per group (>= 1)
     float scale_log2;        // scale * log2(e)
+    // optional (may be null): [0] += (warp, key tile) steps that rescaled O,
+    // [1] += (row, key tile) rescales; counted by the two-query-tile kernel
+    unsigned long long* rescale_stats;
 };
 
 // Load sequence of the K/V ring: K_0 .. K_{min(3,n)-1}, then for each step t
@@ -538,87 +531,58 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // 2m / 2m+1 = keys 8m + kq + {0,1} of row a / row b, which is the
                 // 16x128b store layout at column 4m + t%4 of the P region.
                 uint64_t la2 = 0, lb2 = 0, ha2 = 0, hb2 = 0;
-                float hsa0 = 0.f, hsa1 = 0.f, hsb0 = 0.f, hsb1 = 0.f;
                 uint32_t pk[32];
-                if constexpr (FA_SOFTMAX_PHASED) {
-                    // pass 1: exponents c*s - m, in place
-    #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int m = i >> 1;
-                        const int o = 4 * m + 2 * (i & 1);
-                        const uint64_t x2 = fma2(f2(__uint_as_float(s[o]), __uint_as_float(s[o + 1])), c2,
-                                                 (i & 1) ? negb : nega);
-                        float x0, x1;
-                        f2_split(x2, x0, x1);
-                        s[o] = __float_as_uint(x0);
-                        s[o + 1] = __float_as_uint(x1);
-                    }
-                    // pass 2: exponentials in place
-    #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int o = 4 * (i >> 1) + 2 * (i & 1);
-                        float p0, p1;
-                        if (EMU > 0 && (i % (EMU > 0 ? EMU : 1)) == EMU - 1) {
-                            exp2_poly2(__uint_as_float(s[o]), __uint_as_float(s[o + 1]), p0, p1);
-                        } else {
-                            p0 = ex2_approx(__uint_as_float(s[o]));
-                            p1 = ex2_approx(__uint_as_float(s[o + 1]));
-                        }
-                        s[o] = __float_as_uint(p0);
-                        s[o + 1] = __float_as_uint(p1);
-                    }
-                    // pass 3: bf16 pairs and the two sums
-    #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int o = 4 * (i >> 1) + 2 * (i & 1);
-                        const float p0 = __uint_as_float(s[o]), p1 = __uint_as_float(s[o + 1]);
-                        const uint32_t w = pack_bf16x2(p0, p1);
-                        const uint64_t pr = f2(p0, p1);
-                        const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-                        if (i & 1) {
-                            lb2 = add2(lb2, pr);
-                            hb2 = add2(hb2, ph);
-                        } else {
-                            la2 = add2(la2, pr);
-                            ha2 = add2(ha2, ph);
-                        }
-                        pk[i] = w;
-                    }
-                } else
+                // The exponentials of the tile are evaluated in three passes:
+                // pass 1, exponents c*s - m, in place
     #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int m = i >> 1;
-                    const bool row_b = i & 1;
-                    const uint64_t x2 = fma2(f2(__uint_as_float(s[4 * m + 2 * row_b]),
-                                                __uint_as_float(s[4 * m + 2 * row_b + 1])),
-                                             c2, row_b ? negb : nega);
+                    const int o = 4 * m + 2 * (i & 1);
+                    const uint64_t x2 = fma2(f2(__uint_as_float(s[o]), __uint_as_float(s[o + 1])), c2,
+                                             (i & 1) ? negb : nega);
                     float x0, x1;
                     f2_split(x2, x0, x1);
+                    s[o] = __float_as_uint(x0);
+                    s[o + 1] = __float_as_uint(x1);
+                }
+                // pass 2: exponentials in place
+    #pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int o = 4 * (i >> 1) + 2 * (i & 1);
                     float p0, p1;
                     if (EMU > 0 && (i % (EMU > 0 ? EMU : 1)) == EMU - 1) {
-                        exp2_poly2(x0, x1, p0, p1);
+                        exp2_poly2(__uint_as_float(s[o]), __uint_as_float(s[o + 1]), p0, p1);
                     } else {
-                        p0 = ex2_approx(x0);
-                        p1 = ex2_approx(x1);
+                        p0 = ex2_approx(__uint_as_float(s[o]));
+                        p1 = ex2_approx(__uint_as_float(s[o + 1]));
                     }
+                    s[o] = __float_as_uint(p0);
+                    s[o + 1] = __float_as_uint(p1);
+                }
+                // pass 3: bf16 pairs and the two sums
+    #pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int o = 4 * (i >> 1) + 2 * (i & 1);
+                    const float p0 = __uint_as_float(s[o]), p1 = __uint_as_float(s[o + 1]);
                     const uint32_t w = pack_bf16x2(p0, p1);
                     const uint64_t pr = f2(p0, p1);
-                    if (row_b) lb2 = add2(lb2, pr);
-                    else la2 = add2(la2, pr);
-                    if constexpr (FA_LHAT_MIXED_ADD) {
-                        if (row_b) add_bf16x2_halves(hsb0, hsb1, w);
-                        else add_bf16x2_halves(hsa0, hsa1, w);
+                    const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+                    if (i & 1) {
+                        lb2 = add2(lb2, pr);
+                        hb2 = add2(hb2, ph);
                     } else {
-                        const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-                        if (row_b) hb2 = add2(hb2, ph);
-                        else ha2 = add2(ha2, ph);
+                        la2 = add2(la2, pr);
+                        ha2 = add2(ha2, ph);
                     }
                     pk[i] = w;
                 }
-                // Pin the packed words in registers ahead of the asynchronous
-                // TMEM store.  Without this fence the multi-pass form above was
-                // observed on sm_100a to store stale register contents (the score
-                // tile) instead of P; the fence emits no instruction.
+                // The TMEM store is an asm statement with register inputs, and
+                // neither it nor tcgen05.wait::st below tells the compiler that the
+                // hardware may still read those registers after the statement
+                // issues.  The fences make the packed words fully computed before
+                // the store and keep their registers unreused until the wait
+                // (without them the multi-pass form above stored stale score
+                // values on sm_100a).  They emit no instruction.
                 reg_fence32(pk);
                 tmem_st16x128b_x16(t_s + C::kColP, pk);
                 float u0, u1;
@@ -630,9 +594,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 lh_a += u0 + u1;
                 f2_split(hb2, u0, u1);
                 lh_b += u0 + u1;
-                lh_a += hsa0 + hsa1;
-                lh_b += hsb0 + hsb1;
                 tmem_wait_st();
+                reg_fence32(pk);
                 tc_fence_before();
                 mbar_arrive(bar_p_full + 8 * bb);
             }

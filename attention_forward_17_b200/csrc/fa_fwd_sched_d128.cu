@@ -4,8 +4,10 @@
 // tile takes another 32 KiB, so at most five slots; at least four keep the
 // ring's parity waits sound), plus the two persistent launches and the split-KV ping-pong kernel (P in shared
 // memory, which leaves room for a four-slot ring only) (one CTA per SM
-// walking several query tiles) for the default exponential split.  First
-// entry = default.
+// walking several query tiles) for the default exponential split, and the
+// two-query-tile kernel (Q_0 and Q_1 take 64 KiB, so at most five slots; its
+// ring is sound at any depth) over the exponential split.  First entry =
+// default.
 #include "fa_schedules.h"
 
 namespace fa {
@@ -16,6 +18,8 @@ const Schedule kD128[] = {
     make_schedule<128, 4, 5, 1>(), make_schedule<128, 4, 4, 1>(),
     make_schedule<128, 4, 5, 2>(), make_schedule<128, 4, 4, 2>(),
     make_pp_schedule<128, 4, 4>(), make_pp_schedule<128, 0, 4>(),
+    make_2q_schedule<128, 4, 5>(), make_2q_schedule<128, 8, 5>(), make_2q_schedule<128, 2, 5>(),
+    make_2q_schedule<128, 0, 5>(), make_2q_schedule<128, 4, 3>(),
 };
 }  // namespace
 

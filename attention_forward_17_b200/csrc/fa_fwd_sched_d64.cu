@@ -1,7 +1,8 @@
 // Compiled schedules of the attention kernel for head dimension 64: the
 // exponential split (EMU) times the K/V ring depth (SLOTS, 16 KiB a slot),
-// plus the two persistent launches and the split-KV ping-pong kernel for the default exponential split.  First entry
-// = default.
+// plus the two persistent launches and the split-KV ping-pong kernel for the
+// default exponential split, and the two-query-tile kernel.  First entry =
+// default.
 #include "fa_schedules.h"
 
 namespace fa {
@@ -13,6 +14,8 @@ const Schedule kD64[] = {
     make_schedule<64, 4, 8, 2>(), make_schedule<64, 4, 4, 2>(),
     make_pp_schedule<64, 4, 8>(), make_pp_schedule<64, 4, 4>(),
     make_pp_schedule<64, 0, 8>(),
+    make_2q_schedule<64, 4, 8>(), make_2q_schedule<64, 2, 8>(), make_2q_schedule<64, 0, 8>(),
+    make_2q_schedule<64, 4, 4>(),
 };
 }  // namespace
 

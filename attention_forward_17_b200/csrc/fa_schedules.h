@@ -9,12 +9,15 @@
 
 #include "fa_fwd_kernel.cuh"
 #include "fa_fwd_pp_kernel.cuh"
+#include "fa_fwd_2q_kernel.cuh"
 
 namespace fa {
 
+// tq, tk, tv: the Q, K, V maps; to: the same view of O (used by the kernels
+// that store O with TMA).
 using FwdLaunchFn = cudaError_t (*)(const CUtensorMap& tq, const CUtensorMap& tk,
-                                    const CUtensorMap& tv, const FwdParams& p, unsigned grid,
-                                    cudaStream_t stream);
+                                    const CUtensorMap& tv, const CUtensorMap& to, const FwdParams& p,
+                                    unsigned grid, cudaStream_t stream);
 
 struct Schedule {
     int d;             // head dimension
@@ -23,7 +26,8 @@ struct Schedule {
     int persist;       // launch form: 0 one tile per CTA, 1 persistent (static), 2 persistent by
                        // cluster launch control (tiles taken over from unlaunched CTAs)
     int alg;           // 0: one softmax pass over every key tile; 1: split-KV ping-pong
-                       // (two softmax groups take alternate key tiles, merged at the end)
+                       // (two softmax groups take alternate key tiles, merged at the end);
+                       // 2: two query tiles per CTA, P over S in TMEM, one issuer per tile
     int smem_bytes;    // dynamic shared memory per CTA
     FwdLaunchFn launch[2];   // [causal]
     int (*setup)();          // shared-memory opt-in and register check, both modes
@@ -37,7 +41,7 @@ const Schedule* schedules_d64(int* count);
 // Shared by both definition files.
 template <int D, bool CAUSAL, int EMU, int SLOTS>
 cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                      const FwdParams& p, unsigned grid, cudaStream_t stream) {
+                      const CUtensorMap&, const FwdParams& p, unsigned grid, cudaStream_t stream) {
     fa_fwd_pp_kernel<D, CAUSAL, EMU, SLOTS>
         <<<grid, kThreads, PPCfg<D, SLOTS>::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
@@ -73,9 +77,49 @@ constexpr Schedule make_pp_schedule() {
                     &setup_pp_both<D, EMU, SLOTS>};
 }
 
+template <int D, bool CAUSAL, int EMU, int SLOTS>
+cudaError_t launch_2q(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const CUtensorMap& to, const FwdParams& p, unsigned grid, cudaStream_t stream) {
+    fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS>
+        <<<grid, kThreads, Q2Cfg<D, SLOTS>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+    return cudaGetLastError();
+}
+
+template <int D, bool CAUSAL, int EMU, int SLOTS>
+int setup_2q_one() {
+    auto* k = fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS>;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Q2Cfg<D, SLOTS>::kSmemBytes) != cudaSuccess)
+        return -6;
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, k) != cudaSuccess) return -6;
+    if (attr.numRegs * kThreads < kRegSplitTotal) return -6;
+    return 0;
+}
+
+template <int D, int EMU, int SLOTS>
+int setup_2q_both() {
+    const int rc = setup_2q_one<D, false, EMU, SLOTS>();
+    return rc ? rc : setup_2q_one<D, true, EMU, SLOTS>();
+}
+
+// Two query tiles per CTA (fa_fwd_2q_kernel).
+template <int D, int EMU, int SLOTS>
+constexpr Schedule make_2q_schedule() {
+    return Schedule{D,
+                    EMU,
+                    SLOTS,
+                    0,
+                    2,
+                    Q2Cfg<D, SLOTS>::kSmemBytes,
+                    {&launch_2q<D, false, EMU, SLOTS>, &launch_2q<D, true, EMU, SLOTS>},
+                    &setup_2q_both<D, EMU, SLOTS>};
+}
+
 template <int D, bool CAUSAL, int EMU, int SLOTS, int PERSIST>
 cudaError_t launch_schedule(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const FwdParams& p, unsigned grid, cudaStream_t stream) {
+                            const CUtensorMap&, const FwdParams& p, unsigned grid,
+                            cudaStream_t stream) {
     fa_fwd_kernel<D, CAUSAL, EMU, SLOTS, PERSIST>
         <<<grid, kThreads, TileCfg<D, SLOTS>::kSmemBytes, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();

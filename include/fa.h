@@ -123,7 +123,11 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
  *                     one softmax pass over every key tile, 1 = split-KV
  *                     ping-pong: two softmax warp groups take alternate key
  *                     tiles with their own running statistics and output
- *                     accumulators, merged per row at the end) and shared memory per CTA of
+ *                     accumulators, merged per row at the end; 2 = two
+ *                     128-row query tiles per CTA sharing every key/value
+ *                     tile, P kept over the scores in tensor memory, one
+ *                     tensor-core issuing thread per query tile, O stored
+ *                     through shared memory with TMA) and shared memory per CTA of
  *                     schedule `id`; FA_ERR_ARG for an unknown id.  Output
  *                     pointers may be NULL.
  * fa_fwd_pick_schedule - the schedule id and causal group fa_fwd uses for
@@ -146,6 +150,25 @@ int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float*
                     int causal_group, int* dev_status, void* stream);
 
 /*
+ * fa_fwd_rescale_stats - fa_fwd_schedule (causal_group from the table) that
+ * also counts the lazy rescales of the output accumulator ("rescaling
+ * factors" of the FlashAttention section: a row's O is rescaled only when its
+ * running maximum grew by more than 2^8 since the last rescale).
+ *
+ *   schedule_id  as for fa_fwd_schedule (-1: the table's choice).
+ *   dev_counts   device, two unsigned 64-bit counters, caller-owned, never
+ *                cleared: [0] += (warp, key tile) steps at which at least one
+ *                of the warp's 32 rows rescaled, [1] += (row, key tile)
+ *                rescales.  Only the two-query-tile kernel (algorithm 2)
+ *                counts; other schedules leave the counters unchanged.
+ *                NULL -> FA_ERR_NULL (after the checks of fa_fwd).
+ * A diagnostic entry point: the atomics cost a little time.
+ */
+int fa_fwd_rescale_stats(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+                         int schedule_id, unsigned long long* dev_counts, void* stream);
+
+/*
  * fa_fwd_host - the same computation starting from and ending in host memory.
  *
  * Copies q_h, k_h, v_h (host, bf16 [B,H,N,d]; pinned memory makes the copies
@@ -153,14 +176,17 @@ int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float*
  * forward pass on them into o_d and lse_d; copies o_d and lse_d back into o_h
  * and lse_h (host).  The (b, h) slices are processed in up to eight chunks so
  * that uploads, kernels and downloads of consecutive chunks overlap: the
- * kernels run on `stream`, the copies on two streams the call creates and
- * releases (the runtime frees them once their work is done), ordered by
- * events so that the copies start after all earlier work on `stream` and
- * `stream` completes only after the last download.  Nothing is allocated on
- * the device; the call returns without synchronising, so the host buffers must
- * stay valid until `stream` has completed.  Argument checks are those of
- * fa_fwd applied to the device buffers, plus FA_ERR_NULL for a NULL host
- * pointer; a failure after some work was enqueued returns FA_ERR_CUDA.
+ * kernels run on `stream`, the copies on two copy streams the library creates
+ * once per device (with a few events) and keeps for the life of the process,
+ * ordered by events so that the copies start after all earlier work on
+ * `stream` and `stream` completes only after the last download.  Concurrent
+ * calls on one device take turns enqueueing their copies on those streams.
+ * Nothing is allocated on the device; the call returns without synchronising,
+ * so the host buffers must stay valid until `stream` has completed.  Argument
+ * checks are those of fa_fwd applied to the device buffers, plus FA_ERR_NULL
+ * for a NULL host pointer.  A failure after some work was enqueued returns
+ * FA_ERR_CUDA, and `stream` is still made to wait for every copy that was
+ * queued, so its completion still means no copy touches the host buffers.
  */
 int fa_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o_h, float* lse_h,
                 void* q_d, void* k_d, void* v_d, void* o_d, float* lse_d, int64_t B, int64_t H,

@@ -150,12 +150,15 @@ def test_schedule_registry():
     for i in range(n):
         assert LIB.fa_schedule_info(i, *[ctypes.byref(x) for x in vals]) == fa.FA_OK
         d, emu, slots, persist, alg, smem = (x.value for x in vals)
-        assert d in (64, 128) and emu in (0, 2, 4) and slots >= 4 and persist in (0, 1, 2)
-        assert alg in (0, 1) and 0 < smem <= 232448
+        assert d in (64, 128) and emu in (0, 2, 4, 8) and persist in (0, 1, 2)
+        assert alg in (0, 1, 2) and 0 < smem <= 232448
+        # the one-tile kernels need four slots for sound parity waits; the
+        # two-tile kernel's issuers observe every load in order, so any depth >= 2
+        assert slots >= (2 if alg == 2 else 4)
         assert (d, emu, slots, persist, alg) not in seen
         seen.add((d, emu, slots, persist, alg))
     assert any(k[3] == 1 for k in seen) and any(k[3] == 2 for k in seen)
-    assert any(k[4] == 1 for k in seen)
+    assert any(k[4] == 1 for k in seen) and any(k[4] == 2 and k[0] == d for k in seen for d in (64, 128))
     assert LIB.fa_schedule_info(n, None, None, None, None, None, None) == fa.FA_ERR_ARG
     assert LIB.fa_schedule_info(-1, None, None, None, None, None, None) == fa.FA_ERR_ARG
     # the first schedule of each head dimension is the default
@@ -181,6 +184,15 @@ def test_schedule_argument_checks():
     assert LIB.fa_fwd_pick_schedule(4096, 128, 1, None, ctypes.byref(grp)) == fa.FA_ERR_NULL
     assert LIB.fa_fwd_pick_schedule(-1, 128, 1, ctypes.byref(sid), ctypes.byref(grp)) == fa.FA_ERR_SHAPE
     assert LIB.fa_fwd_pick_schedule(64, 80, 1, ctypes.byref(sid), ctypes.byref(grp)) == fa.FA_ERR_HEADDIM
+
+
+def test_rescale_stats_argument_checks():
+    f = LIB.fa_fwd_rescale_stats
+    args = (16, 32, 48, 64, 80, 1, 1, 128, 128, 0, 0.125)
+    assert f(*args, -1, None, None) == fa.FA_ERR_NULL          # counters required
+    assert f(*args, -2, 96, None) == fa.FA_ERR_ARG             # schedule id below -1
+    assert f(*args[:5], 0, 1, 128, 128, 0, 0.125, -1, None, None) == fa.FA_OK     # empty: no-op
+    assert f(*args[:8], 80, 0, 0.125, -1, 96, None) == fa.FA_ERR_HEADDIM          # fa_fwd's checks first
 
 
 def test_launch_count():

@@ -65,3 +65,27 @@ def test_schedule_report_respects_pins():
     assert pinned["id"] == 0 and pinned["causal_group"] == 3
     assert auto["id"] >= 0 and "algorithm" in auto
     assert bench.schedule_of(4096, 64, False)["causal_group"] is None
+
+
+def test_sample_parity_checks_all_three_bars():
+    import numpy as np
+    import torch
+    rng = np.random.default_rng(0)
+    d, n = 8, 40
+    o_ref = rng.standard_normal((n, d))
+    lse_ref = rng.standard_normal(n)
+    rows = np.arange(n)
+    o = torch.tensor(o_ref, dtype=torch.float32).to(torch.bfloat16).view(1, 1, n, d)
+    lse = torch.tensor(lse_ref, dtype=torch.float32).view(1, 1, n)
+    res = [(rows, {False: (o_ref, lse_ref)})]
+    good = bench.sample_parity(res, {False: o}, {False: lse}, d)
+    assert good["pass"] and good["o_rel_l2"] < 1e-2
+    # a uniform 1.5 % relative error stays under the max-abs bar (|O| <= ~1.3 here)
+    # but fails the relative-L2 bar
+    far = torch.tensor(o_ref * 1.015, dtype=torch.float32).view(1, 1, n, d)
+    o_ref_small = o_ref * (0.01 / np.abs(o_ref).max())
+    res_small = [(rows, {False: (o_ref_small, lse_ref)})]
+    bad = bench.sample_parity(res_small, {False: torch.tensor(o_ref_small * 1.015).view(1, 1, n, d)},
+                              {False: lse}, d)
+    assert bad["o_max_abs"] <= 2e-2 and bad["o_rel_l2"] > 1e-2 and not bad["pass"]
+    assert not bench.sample_parity(res, {False: far}, {False: lse + 0.01}, d)["pass"]

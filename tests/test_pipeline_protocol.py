@@ -25,6 +25,19 @@ tile per CTA).
 This is the reasoning that found a real race (the output issuer used to wait
 for V_t before P_t); the last tests check that the model flags that order and
 a three-slot ring.
+
+The two-query-tile kernel (algorithm 2) loads K_0, V_0, K_1, V_1, ... once for
+both of its query tiles, and each of its two issuers visits every load in that
+order: it waits for the load to land and then uses it (products, then a
+release by commit) or, for key tiles its query tile does not need under the
+causal mask, releases it by a plain arrival.  Each release needs both issuers.
+Two things must hold: a parity wait on load i starts after the waiter observed
+load i - SLOTS (true when every visit waits, in order), and a release arrival
+for load i lands in load i's phase of the slot's empty barrier, which holds
+once load i has landed (the producer issued it after load i - SLOTS was
+released by both issuers).  The model below checks both for every compiled
+depth and every pair of key-tile counts, and flags an issuer that releases
+unused loads without waiting for them.
 """
 import random
 
@@ -73,7 +86,7 @@ def violations(tiles, slots, algorithm, v_before_p=False):
 
 
 def compiled_rings():
-    return sorted({(s["kv_slots"], s["algorithm"]) for s in fa.schedules()})
+    return sorted({(s["kv_slots"], s["algorithm"]) for s in fa.schedules() if s["algorithm"] != 2})
 
 
 def compiled_multi_tile_rings():
@@ -119,3 +132,83 @@ def test_model_flags_an_odd_ring_for_the_ping_pong_kernel():
     # slot predecessor must itself be a K tile: odd depths break that
     assert sum(violations([n], 5, 1) for n in range(1, 40)) > 0
     assert all(s["kv_slots"] % 2 == 0 for s in fa.schedules() if s["algorithm"] == 1)
+
+
+# ------------------------------------------------------------------ two-query-tile kernel
+def two_tile_issuer_events(n0, n1, release_k_early=False):
+    """The ring events of the two-query-tile kernel's single MMA issuer, in
+    program order, for key-tile counts n0 (tile 0) and n1 (tile 1): ("wait", L),
+    ("use", L), ("release", L) with L the load index (K_j = 2j, V_j = 2j+1).
+    release_k_early models a faulty variant that releases K_{j+1} right after
+    tile 0's score product."""
+    ev, waited = [], [-1]
+
+    def wait(ld):
+        if ld > waited[0]:
+            ev.append(("wait", ld))
+            waited[0] = ld
+
+    n_kv = max(n0, n1)
+    wait(0)
+    ev.append(("use", 0))
+    if n1 > 0:
+        ev.append(("use", 0))
+    ev.append(("release", 0))
+    for j in range(n_kv):
+        for ti, n_i in ((0, n0), (1, n1)):
+            if j >= n_i:
+                continue
+            wait(2 * j + 1)
+            ev.append(("use", 2 * j + 1))
+            if j + 1 < n_i:
+                wait(2 * j + 2)
+                ev.append(("use", 2 * j + 2))
+                if release_k_early and ti == 0:
+                    ev.append(("release", 2 * j + 2))
+        ev.append(("release", 2 * j + 1))
+        if j + 1 < n_kv and not (release_k_early and j + 1 < n0):
+            ev.append(("release", 2 * j + 2))
+    return ev, 2 * n_kv
+
+
+def two_tile_violations(n0, n1, slots, **kw):
+    """Unsound parity waits, uses of unobserved or released loads, and loads
+    released twice or never, for the issuer's event sequence."""
+    ev, loads = two_tile_issuer_events(n0, n1, **kw)
+    bad = 0
+    landed, released = set(), set()
+    for kind, ld in ev:
+        if kind == "wait":
+            # a parity wait on load ld is sound once the slot's previous load was observed
+            if ld >= slots and (ld - slots) not in landed:
+                bad += 1
+            landed.add(ld)
+        elif kind == "use":
+            if ld not in landed or ld in released:
+                bad += 1
+        else:
+            if ld not in landed or ld in released:
+                bad += 1
+            released.add(ld)
+    # the producer reuses a slot after the release of its previous load: every load must be released
+    bad += loads - len(released)
+    return bad
+
+
+def compiled_two_tile_depths():
+    return sorted({s["kv_slots"] for s in fa.schedules() if s["algorithm"] == 2})
+
+
+@pytest.mark.parametrize("slots", compiled_two_tile_depths())
+def test_two_tile_ring_is_sound(slots):
+    for n1 in range(0, 40):
+        # non-causal (equal counts), causal (tile 0 one key tile short), and a
+        # second tile past the end of the sequence (no keys)
+        for n0 in {n1, n1 - 1}:
+            if n0 >= 1:
+                assert two_tile_violations(n0, n1, slots) == 0, (n0, n1)
+        assert two_tile_violations(n1 + 1, 0, slots) == 0
+
+
+def test_model_flags_an_early_key_release():
+    assert sum(two_tile_violations(n, n, 5, release_k_early=True) for n in range(2, 20)) > 0

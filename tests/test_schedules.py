@@ -6,15 +6,18 @@ with several tiles per CTA, and the table's choice for each problem class."""
 import numpy as np
 import pytest
 
+import attention_forward_17_b200 as fa_lib
 import oracle
 import parity_utils as pu
 
 pytestmark = pytest.mark.gpu
 
+# the library loads without a GPU, so the compiled schedules are known at collection
+N_SCHEDULES = fa_lib.lib.fa_schedule_count()
+
 
 def _schedules():
-    import attention_forward_17_b200 as fa
-    return fa.schedules()
+    return fa_lib.schedules()
 
 
 def run_sched(qt, kt, vt, causal, sid, group):
@@ -25,11 +28,9 @@ def run_sched(qt, kt, vt, causal, sid, group):
     return pu.o_f64(o), lse.double().cpu().numpy()
 
 
-@pytest.mark.parametrize("sid", range(32))
+@pytest.mark.parametrize("sid", range(N_SCHEDULES))
 def test_every_schedule_matches_oracle(cuda_device, sid):
     sched = _schedules()
-    if sid >= len(sched):
-        pytest.skip("fewer schedules compiled")
     d = sched[sid]["d"]
     (q, k, v), (qt, kt, vt) = pu.inputs(1, 2, 1000, d, seed=sid, sigma_qk=3.0)
     for causal in (False, True):
@@ -67,14 +68,22 @@ def test_persistent_walks_every_tile(cuda_device, d, N):
             pu.check(o, lse, o_ref, lse_ref, f"persistent {s} causal={causal} N={N}")
 
 
-def test_table_choice_is_valid():
-    import attention_forward_17_b200 as fa
-    sched = fa.schedules()
-    for d in (64, 128):
-        for causal in (False, True):
-            for N in (1, 1024, 2048, 2049, 4096, 8193, 16384, 1 << 20):
-                sid, grp = fa.pick_schedule(N, d, causal)
-                assert 0 <= sid < len(sched) and sched[sid]["d"] == d and grp >= 1
+@pytest.mark.gpu
+def test_two_tile_kernel_edges(cuda_device):
+    # the two-query-tile kernel on shapes that exercise its pairing: one row, a
+    # lone first tile, a pair whose second tile is ragged or empty (odd tile
+    # counts), several slices, both masks
+    sched = [s for s in _schedules() if s["algorithm"] == 2]
+    assert sched, "no two-query-tile schedule compiled"
+    for s in sched:
+        d = s["d"]
+        for B, H, N in ((1, 1, 1), (1, 2, 100), (1, 1, 129), (2, 1, 255), (1, 3, 256), (1, 2, 257),
+                        (1, 1, 385), (2, 2, 640)):
+            (q, k, v), (qt, kt, vt) = pu.inputs(B, H, N, d, seed=N + d, sigma_qk=3.0)
+            for causal in (False, True):
+                o_ref, lse_ref = oracle.attention_fwd(q, k, v, causal, pu.default_scale(d))
+                o, lse = run_sched(qt, kt, vt, causal, s["id"], 1)
+                pu.check(o, lse, o_ref, lse_ref, f"two-tile {s} B{B} H{H} N{N} causal={causal}")
 
 
 def test_default_path_uses_the_table_choice(cuda_device):
