@@ -5,10 +5,10 @@ from ._binding import (FA_ERR_ALIGN, FA_ERR_ARCH, FA_ERR_ARG, FA_ERR_CUDA, FA_ER
                        FA_ERR_NULL, FA_ERR_SCALE, FA_ERR_SHAPE, FA_ERR_TIMEOUT, FA_GEMM_BIAS,
                        FA_GEMM_BIAS_GELU, FA_GEMM_PLAIN, FA_OK, FaError, LIB_PATH, fa_fwd,
                        fa_fwd_host, gemm, header_functions, launches_per_call, lib, pick_schedule,
-                       row_softmax, schedules, selftest_wait_timeout, strerror, vector_add,
+                       rescale_stats, row_softmax, schedules, selftest_wait_timeout, strerror, vector_add,
                        version)
 
-__all__ = ["fa_fwd", "fa_fwd_host", "row_softmax", "gemm", "vector_add", "schedules",
+__all__ = ["fa_fwd", "fa_fwd_host", "rescale_stats", "row_softmax", "gemm", "vector_add", "schedules",
            "pick_schedule", "selftest_wait_timeout",
            "FaError", "strerror", "version", "launches_per_call", "header_functions", "lib",
            "LIB_PATH", "FA_OK", "FA_ERR_NULL", "FA_ERR_SHAPE", "FA_ERR_HEADDIM", "FA_ERR_ALIGN",

@@ -70,7 +70,7 @@ def _load():
     lib.fa_fwd_rescale_stats.restype = ctypes.c_int
     lib.fa_schedule_count.argtypes = []
     lib.fa_schedule_count.restype = ctypes.c_int
-    lib.fa_schedule_info.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp]
+    lib.fa_schedule_info.argtypes = [ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     lib.fa_schedule_info.restype = ctypes.c_int
     lib.fa_fwd_pick_schedule.argtypes = [_i64, _i64, ctypes.c_int, _vp, _vp]
     lib.fa_fwd_pick_schedule.restype = ctypes.c_int
@@ -133,16 +133,16 @@ def _check_qkv(q, k, v):
 
 def schedules() -> list[dict]:
     """Every compiled schedule of the attention kernel: id, d, emu_every, kv_slots,
-    persistent, algorithm, smem_bytes."""
+    persistent, algorithm, smem_bytes, key_tile."""
     out = []
     for i in range(lib.fa_schedule_count()):
-        vals = [ctypes.c_int() for _ in range(6)]
+        vals = [ctypes.c_int() for _ in range(7)]
         rc = lib.fa_schedule_info(i, *[ctypes.byref(x) for x in vals])
         if rc != FA_OK:
             raise FaError(rc, "fa_schedule_info")
         out.append(dict(id=i, d=vals[0].value, emu_every=vals[1].value, kv_slots=vals[2].value,
                         persistent=vals[3].value, algorithm=vals[4].value,
-                        smem_bytes=vals[5].value))
+                        smem_bytes=vals[5].value, key_tile=vals[6].value))
     return out
 
 

@@ -113,7 +113,7 @@ int device_setup(int dev) {
 // The schedule id fa_fwd uses for (N, d, causal), and the causal launch group.
 void pick_schedule(int64_t N, int64_t d, int causal, int* id, int* group) {
     const ScheduleList& list = schedules();
-    int emu = -1, slots = -1, grp = 1, persist = 0, alg = 0;
+    int emu = -1, slots = -1, grp = 1, persist = 0, alg = 0, bn = 128;
     for (const auto& e : fa::kScheduleTable)
         if (e.d == d && e.causal == (causal ? 1 : 0) && N <= e.n_max) {
             emu = e.emu;
@@ -121,19 +121,21 @@ void pick_schedule(int64_t N, int64_t d, int causal, int* id, int* group) {
             grp = e.group;
             persist = e.persist;
             alg = e.alg;
+            bn = e.bn;
             break;
         }
-    int first = -1, match = -1;
+    int match = -1;
     for (int i = 0; i < list.count; ++i) {
         const fa::Schedule* s = list.items[i];
-        if (s->d != d) continue;
-        if (first < 0) first = i;
-        if (s->emu == emu && s->slots == slots && s->persist == persist && s->alg == alg) {
+        if (s->d == d && s->emu == emu && s->slots == slots && s->persist == persist &&
+            s->alg == alg && s->bn == bn) {
             match = i;
             break;
         }
     }
-    *id = match >= 0 ? match : first;
+    // -1 when the table names a schedule that is not compiled (a build
+    // inconsistency that the tests rule out; run_fwd then refuses to launch)
+    *id = match;
     *group = grp > 0 ? grp : 1;
 }
 
@@ -157,13 +159,15 @@ int encoder_ready() {
     return g_encode ? FA_OK : FA_ERR_CUDA;
 }
 
-// 3-D view [BH][N][d] of a bf16 tensor; boxes of 128 rows x 64 columns
-// (128 bytes, matching the 128-byte swizzle); rows past N read as zero.
-int encode_qkv_map(CUtensorMap* map, const void* ptr, int64_t BH, int64_t N, int64_t d) {
+// 3-D view [BH][N][d] of a bf16 tensor; boxes of `rows` rows x 64 columns
+// (128 bytes, matching the 128-byte swizzle); rows past N read as zero and
+// are not written by stores.
+int encode_qkv_map(CUtensorMap* map, const void* ptr, int64_t BH, int64_t N, int64_t d,
+                   uint32_t rows = 128) {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                           static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * 2), static_cast<cuuint64_t>(N * d * 2)};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, rows, 1};
     cuuint32_t elem[3] = {1, 1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                           strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -205,14 +209,18 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
     int table_id = 0, table_group = 1;
     pick_schedule(N, d, causal, &table_id, &table_group);
     if (schedule_id < 0) schedule_id = table_id;
+    if (schedule_id < 0) return FA_ERR_ARG;
     if (group < 1) group = table_group;
     int sms = 0;
     if ((rc = current_device_ready(&sms)) != FA_OK) return rc;
     if ((rc = encoder_ready()) != FA_OK) return rc;
     const int64_t BH = B * H;
+    const fa::Schedule* sch = list.items[schedule_id];
+    // K and V boxes are one key tile (sch->bn rows); Q and O boxes one 128-row query tile
     alignas(64) CUtensorMap tq, tk, tv, to;
-    if (encode_qkv_map(&tq, q, BH, N, d) || encode_qkv_map(&tk, k, BH, N, d) ||
-        encode_qkv_map(&tv, v, BH, N, d) || encode_qkv_map(&to, o, BH, N, d))
+    const uint32_t bn = static_cast<uint32_t>(sch->bn);
+    if (encode_qkv_map(&tq, q, BH, N, d) || encode_qkv_map(&tk, k, BH, N, d, bn) ||
+        encode_qkv_map(&tv, v, BH, N, d, bn) || encode_qkv_map(&to, o, BH, N, d))
         return FA_ERR_CUDA;
     fa::FwdParams p;
     p.o = static_cast<__nv_bfloat16*>(o);
@@ -226,7 +234,6 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
     p.rescale_stats = rescale_stats;
     int64_t grid = BH * p.n_qtile;
     if (grid > 0x7fffffffLL) return FA_ERR_SHAPE;
-    const fa::Schedule* sch = list.items[schedule_id];
     if (sch->alg == 2) {
         // two query tiles per CTA
         grid = BH * ((p.n_qtile + 1) / 2);
@@ -281,7 +288,7 @@ int fa_fwd_rescale_stats(const void* q, const void* k, const void* v, void* o, f
 int fa_schedule_count(void) { return schedules().count; }
 
 int fa_schedule_info(int id, int* d, int* emu_every, int* kv_slots, int* persistent,
-                     int* algorithm, int* smem_bytes) {
+                     int* algorithm, int* smem_bytes, int* key_tile) {
     const ScheduleList& list = schedules();
     if (id < 0 || id >= list.count) return FA_ERR_ARG;
     const fa::Schedule* s = list.items[id];
@@ -291,6 +298,7 @@ int fa_schedule_info(int id, int* d, int* emu_every, int* kv_slots, int* persist
     if (persistent) *persistent = s->persist;
     if (algorithm) *algorithm = s->alg;
     if (smem_bytes) *smem_bytes = s->smem_bytes;
+    if (key_tile) *key_tile = s->bn;
     return FA_OK;
 }
 
@@ -418,6 +426,6 @@ const char* fa_strerror(int status) {
     }
 }
 
-int fa_version(void) { return (1 << 16) | 1; }
+int fa_version(void) { return (1 << 16) | 2; }
 
 }  // extern "C"

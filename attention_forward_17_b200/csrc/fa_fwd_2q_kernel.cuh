@@ -19,10 +19,13 @@
 //              both tiles, in a fixed alternating order.
 //   warp 10    allocates and frees TMEM.
 //
-// Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
-// O_1 [256+D,256+2D).  The softmax writes P_i (bf16, two keys per column) over
-// columns [64,128) of S_i, and O_i += P_i V_j reads P_i straight from TMEM (the
-// tensor core's TMEM-A form), so P never touches shared memory.
+// Key tiles are BN rows (BN = 64, 128 or 192, a template parameter; the tile
+// of queries is always 128 rows).  Tensor memory (512 columns): S_0 [0,BN),
+// S_1 [BN,2BN), O_0 [2BN,2BN+D), O_1 [2BN+D,2BN+2D), which bounds BN by
+// 2 BN + 2 D <= 512.  The softmax writes P_i (bf16, two keys per column) over
+// the first BN/2 columns of S_i once it has read them, and O_i += P_i V_j reads
+// P_i straight from TMEM (the tensor core's TMEM-A form), so P never touches
+// shared memory.
 //
 // Why a single issuing thread: tcgen05 operations of one thread complete in
 // issue order, and an mbarrier commit fires once every earlier operation of
@@ -51,8 +54,9 @@
 // tensor map): coalesced full-line writes.  LSE (one fp32 per row, consecutive
 // rows in consecutive lanes) is stored directly.
 //
-// Causal mask: tile 0 of pair c needs key tiles 0..2c, tile 1 needs 0..2c+1;
-// the ring carries 2c+2 key tiles and the last one only feeds tile 1.  The
+// Causal mask: query tile i of pair c needs the key tiles that hold keys
+// 0 .. 256c + 128i + 127; the ring carries those of tile 1 and the last ones
+// only feed tile 1.  The
 // issuer waits for every ring load exactly once, in load order, which keeps
 // every parity wait on the ring sound for any depth (it waits for load L only
 // after observing load L-1), and releases each load by one commit after its
@@ -65,23 +69,29 @@
 
 namespace fa {
 
-template <int D, int SLOTS>
+template <int D, int SLOTS, int BN>
 struct Q2Cfg {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    static_assert(BN == 64 || BN == 128 || BN == 192, "key tile of 64, 128 or 192 rows");
     static_assert(SLOTS >= 2, "K/V ring depth");
-    static constexpr int kTileBytes = 128 * D * 2;          // one 128-row tile of Q, K, V or O
+    static constexpr int kQTileBytes = 128 * D * 2;         // one 128-row tile of Q (or O)
+    static constexpr int kKVTileBytes = BN * D * 2;         // one BN-row tile of K or V
     static constexpr int kBoxes = D / 64;                   // 64-column (128-byte) TMA boxes
-    static constexpr int kBoxBytes = 128 * 128;
+    static constexpr int kQBoxBytes = 128 * 128;
+    static constexpr int kKVBoxBytes = BN * 128;
     static constexpr int kSlots = SLOTS;
     static constexpr int kQOff = 0;                         // Q_0, then Q_1 (O staging at the end)
-    static constexpr int kSlotOff = 2 * kTileBytes;
-    static constexpr int kBarOff = kSlotOff + SLOTS * kTileBytes;
+    static constexpr int kSlotOff = 2 * kQTileBytes;
+    static constexpr int kBarOff = kSlotOff + SLOTS * kKVTileBytes;
     static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBarOff + 512;
-    static constexpr uint32_t kColO = 256;
-    static constexpr uint32_t kColP = 64;                   // P_i inside S_i
+    // TMEM: S_0 [0,BN), S_1 [BN,2BN), O_0 [2BN,2BN+D), O_1 [2BN+D,2BN+2D); P_i
+    // (bf16 pairs, BN/2 columns) over the first columns of S_i
+    static constexpr uint32_t kColO = 2 * BN;
     static constexpr uint32_t kTmemCols = 512;
+    static constexpr int kHalfWords = BN / 4;               // P words released at a time
     static_assert(kSmemBytes <= 232448, "shared memory per CTA (227 KiB)");
     static_assert(kColO + 2 * D <= kTmemCols, "two score and two output buffers in TMEM");
+    static_assert(kKVBoxBytes % 1024 == 0, "slots on 1024-byte boundaries (128-byte swizzle)");
 };
 
 template <int kSlots>
@@ -90,11 +100,32 @@ struct alignas(8) Q2Barriers {
     uint64_t kv_empty[kSlots];     // released by one commit after the load's last use
     uint64_t q_full[2];
     uint64_t s_full[2];            // S_i(j) computed (and PV_i(j-1) completed)
-    uint64_t p_full[2];            // P_i(j) in TMEM, O_i rescaled (128 arrivals)
+    uint64_t p_half[2];            // first half of P_i(j)'s keys in TMEM, O_i rescaled (128 arrivals)
+    uint64_t p_full[2];            // second half of P_i(j)'s keys in TMEM (128 arrivals)
     uint64_t o_full[2];            // every product of tile i completed
     uint32_t tmem_base;
     volatile uint32_t abort;
 };
+
+// Stores N words of this thread's TMEM lane at consecutive columns from
+// taddr and waits until the stores completed.  The fences keep the words fully
+// computed before the asynchronous store and their registers untouched until
+// the wait (neither asm statement tells the compiler that the hardware reads
+// the registers after the store issues).
+template <int N>
+__device__ __forceinline__ void store_words(uint32_t taddr, uint32_t (&w)[N]) {
+    static_assert(N % 16 == 0, "whole 16-column stores");
+#pragma unroll
+    for (int q = 0; q < N / 32; ++q) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&w[32 * q]));
+    if constexpr (N % 32) reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&w[N - 16]));
+#pragma unroll
+    for (int q = 0; q < N / 32; ++q) tmem_st32(taddr + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&w[32 * q]));
+    if constexpr (N % 32) tmem_st16(taddr + N - 16, *reinterpret_cast<uint32_t(*)[16]>(&w[N - 16]));
+    tmem_wait_st();
+#pragma unroll
+    for (int q = 0; q < N / 32; ++q) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&w[32 * q]));
+    if constexpr (N % 32) reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&w[N - 16]));
+}
 
 constexpr int kQ2IssuerWarp = 9;       // issues every tcgen05.mma of the CTA
 constexpr int kQ2AllocWarp = 10;
@@ -118,12 +149,12 @@ __device__ __forceinline__ void map_pair(const FwdParams& p, int n_pair, int id,
     }
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                      const FwdParams p) {
-    using C = Q2Cfg<D, SLOTS>;
+    using C = Q2Cfg<D, SLOTS, BN>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -135,12 +166,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_pair = (p.n_qtile + 1) / 2;
     int bh, c;
     map_pair<CAUSAL>(p, n_pair, blockIdx.x, bh, c);
-    const int n_kv_all = (p.N + kBlockN - 1) / kBlockN;
-    // key tiles of query tile i (0 when the tile lies past N)
+    const int n_kv_all = (p.N + BN - 1) / BN;
+    // key tiles of query tile i (0 when the tile lies past N); under the mask
+    // the tiles holding keys 0 .. q0+127
     const auto kv_tiles = [&](int i) {
         const int q0 = 256 * c + 128 * i;
         if (q0 >= p.N) return 0;
-        return CAUSAL ? min(n_kv_all, 2 * c + i + 1) : n_kv_all;
+        return CAUSAL ? min(n_kv_all, (q0 + 128 + BN - 1) / BN) : n_kv_all;
     };
     const int n_kv = max(kv_tiles(0), kv_tiles(1));
 
@@ -148,6 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_kv_empty = smem_u32(&bars->kv_empty[0]);
     const uint32_t bar_q_full = smem_u32(&bars->q_full[0]);
     const uint32_t bar_s_full = smem_u32(&bars->s_full[0]);
+    const uint32_t bar_p_half = smem_u32(&bars->p_half[0]);
     const uint32_t bar_p_full = smem_u32(&bars->p_full[0]);
     const uint32_t bar_o_full = smem_u32(&bars->o_full[0]);
     volatile uint32_t* abort = &bars->abort;
@@ -160,6 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_q_full + 8 * i, 1);
             mbar_init(bar_s_full + 8 * i, 1);
+            mbar_init(bar_p_half + 8 * i, 128);
             mbar_init(bar_p_full + 8 * i, 128);
             mbar_init(bar_o_full + 8 * i, 1);
         }
@@ -191,56 +225,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = q0 + r;
         const int n_i = kv_tiles(ti);
         const uint32_t lane_w = static_cast<uint32_t>(32 * quarter) << 16;
-        const uint32_t t_s = tmem + lane_w + 128u * ti;
-        const uint32_t t_p = t_s + C::kColP;
+        const uint32_t t_s = tmem + lane_w + static_cast<uint32_t>(BN) * ti;
+        const uint32_t t_p = t_s;
         const uint32_t t_o = tmem + lane_w + C::kColO + static_cast<uint32_t>(D) * ti;
         const float cl = p.scale_log2;
         const uint64_t c2 = f2(cl, cl);
         const uint32_t bar_s = bar_s_full + 8 * ti, bar_p = bar_p_full + 8 * ti;
+        const uint32_t bar_ph = bar_p_half + 8 * ti;
 
         float m = -INFINITY;                      // running max of c*s (stale by < 8)
         float l = 0.f, lh = 0.f;                  // sums of the weights: fp32, and bf16-rounded
         for (int j = 0; j < n_i; ++j) {
             wait_bar(bar_s, j & 1, abort, p.status);
             tc_fence_after();
-            uint32_t s[128];
-            {
-                uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
-                uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-                uint32_t (&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[64]);
-                uint32_t (&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[96]);
-                tmem_ld32(t_s, s0);
-                tmem_ld32(t_s + 32, s1);
-                tmem_ld32(t_s + 64, s2);
-                tmem_ld32(t_s + 96, s3);
+            const bool masked =
+                (j * BN + BN > p.N) || (CAUSAL && j * BN + BN - 1 > q0);
+            const int lim = (CAUSAL ? min(p.N, row + 1) : p.N) - j * BN;   // keys >= lim are masked
+            // Scores of this row, 32 columns at a time (kRegCols held in
+            // registers; wider key tiles are read twice: once for the maximum,
+            // once for the exponentials).
+            constexpr int kRegCols = BN <= 128 ? BN : BN / 2;
+            uint32_t s[kRegCols];
+            const auto load_cols = [&](int c0) {
+#pragma unroll
+                for (int q = 0; q < kRegCols / 32; ++q)
+                    tmem_ld32(t_s + c0 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * q]));
                 tmem_wait_ld();
                 // the wait carries no register operands: pin the loaded values after it
-                reg_fence32(s0);
-                reg_fence32(s1);
-                reg_fence32(s2);
-                reg_fence32(s3);
-            }
-            const bool masked =
-                (j * kBlockN + kBlockN > p.N) || (CAUSAL && j * kBlockN + kBlockN - 1 > q0);
-            if (masked) {
-                const int lim = (CAUSAL ? min(p.N, row + 1) : p.N) - j * kBlockN;
 #pragma unroll
-                for (int k = 0; k < 128; ++k)
-                    if (k >= lim) s[k] = __float_as_uint(-INFINITY);
-            }
-            // row maximum: four independent chains of three-way maxima
-            float x0 = fmaxf(__uint_as_float(s[0]), __uint_as_float(s[1]));
-            float x1 = fmaxf(__uint_as_float(s[2]), __uint_as_float(s[3]));
-            float x2 = fmaxf(__uint_as_float(s[4]), __uint_as_float(s[5]));
-            float x3 = fmaxf(__uint_as_float(s[6]), __uint_as_float(s[7]));
+                for (int q = 0; q < kRegCols / 32; ++q)
+                    reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[32 * q]));
+                if (masked) {
 #pragma unroll
-            for (int k = 8; k < 128; k += 8) {
-                x0 = max3f(x0, __uint_as_float(s[k]), __uint_as_float(s[k + 1]));
-                x1 = max3f(x1, __uint_as_float(s[k + 2]), __uint_as_float(s[k + 3]));
-                x2 = max3f(x2, __uint_as_float(s[k + 4]), __uint_as_float(s[k + 5]));
-                x3 = max3f(x3, __uint_as_float(s[k + 6]), __uint_as_float(s[k + 7]));
+                    for (int k = 0; k < kRegCols; ++k)
+                        if (c0 + k >= lim) s[k] = __float_as_uint(-INFINITY);
+                }
+            };
+            // row maximum: independent chains of three-way maxima over 16 keys each,
+            // then a short tree
+            float x[8];
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) x[ch] = -INFINITY;
+#pragma unroll
+            for (int c0 = 0; c0 < BN; c0 += kRegCols) {
+                if (BN > 128 || c0 == 0) load_cols(c0);
+#pragma unroll
+                for (int ch = 0; ch < kRegCols / 16; ++ch) {
+                    float& xc = x[(c0 / 16 + ch) & 7];
+#pragma unroll
+                    for (int k = 0; k < 16; k += 2)
+                        xc = max3f(xc, __uint_as_float(s[16 * ch + k]), __uint_as_float(s[16 * ch + k + 1]));
+                }
             }
-            const float mn = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)) * cl;
+            const float mn =
+                fmaxf(max3f(x[0], x[1], x[2]), max3f(x[3], x[4], fmaxf(x[5], max3f(x[6], x[7], x[7])))) * cl;
             const bool grow = mn > m + 8.0f;
             float alpha = 1.f;
             if (grow) {
@@ -249,75 +287,76 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l *= alpha;
                 lh *= alpha;
             }
+            // Lazy rescale of this row of O_i (O_i holds the products of steps
+            // < j, all completed: S_i(j) was issued after PV_i(j-1)).  The stores
+            // complete before the first release of P below (tcgen05.wait::st).
+            const bool need = grow && j > 0;
+            if (__any_sync(0xffffffffu, need)) {
+                const unsigned rows = __popc(__ballot_sync(0xffffffffu, need));
+                if (p.rescale_stats && lane == 0) {
+                    atomicAdd(p.rescale_stats, 1ull);
+                    atomicAdd(p.rescale_stats + 1, static_cast<unsigned long long>(rows));
+                }
+                __syncwarp();       // the TMEM accesses below are warp-collective
+#pragma unroll 1
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t o[32];
+                    tmem_ld32(t_o + 32 * q, o);
+                    tmem_wait_ld();
+                    reg_fence32(o);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    reg_fence32(o);
+                    tmem_st32(t_o + 32 * q, o);
+                }
+            }
             const float u = (m == -INFINITY) ? 0.f : m;
             const uint64_t negm = f2(-u, -u);
-            // weights 2^(c*s - m), their sums, and P as bf16 pairs: word k = keys 2k, 2k+1
-            uint64_t la0 = 0, la1 = 0, ha0 = 0, ha1 = 0;
-            uint32_t pw[64];
+            // Weights 2^(c*s - m), their sums, and P as bf16 pairs (word k = keys
+            // 2k, 2k+1), in two halves of BN/2 keys: each half is stored to TMEM
+            // and released on its own barrier, so the product with the first
+            // half runs while the second half is computed.  P goes over the
+            // first BN/2 columns of S_i, whose scores this thread has already read.
+            constexpr int kHW = C::kHalfWords;
+            uint64_t la0 = 0, la1 = 0;
+            float hl0 = 0.f, hh0 = 0.f, hl1 = 0.f, hh1 = 0.f;
 #pragma unroll
-            for (int k = 0; k < 64; ++k) {
-                const uint64_t x2v = fma2(f2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), c2, negm);
-                float e0, e1, p0, p1;
-                f2_split(x2v, e0, e1);
-                if (EMU > 0 && (k % (EMU > 0 ? EMU : 1)) == EMU - 1) {
-                    exp2_poly2(e0, e1, p0, p1);
-                } else {
-                    p0 = ex2_approx(e0);
-                    p1 = ex2_approx(e1);
-                }
-                const uint32_t w = pack_bf16x2(p0, p1);
-                const uint64_t pr = f2(p0, p1);
-                const uint64_t ph = f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-                if (k & 1) {
-                    la1 = add2(la1, pr);
-                    ha1 = add2(ha1, ph);
-                } else {
-                    la0 = add2(la0, pr);
-                    ha0 = add2(ha0, ph);
-                }
-                pw[k] = w;
-            }
-            {
-                uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pw[0]);
-                uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pw[32]);
-                reg_fence32(p0);
-                reg_fence32(p1);
-                tmem_st32(t_p, p0);
-                tmem_st32(t_p + 32, p1);
-                // Lazy rescale of this row of O_i (O_i holds the products of steps
-                // < j, all completed: S_i(j) was issued after PV_i(j-1)).
-                const bool need = grow && j > 0;
-                if (__any_sync(0xffffffffu, need)) {
-                    const unsigned rows = __popc(__ballot_sync(0xffffffffu, need));
-                    if (p.rescale_stats && lane == 0) {
-                        atomicAdd(p.rescale_stats, 1ull);
-                        atomicAdd(p.rescale_stats + 1, static_cast<unsigned long long>(rows));
-                    }
-                    __syncwarp();       // the TMEM accesses below are warp-collective
-#pragma unroll 1
-                    for (int q = 0; q < D / 32; ++q) {
-                        uint32_t o[32];
-                        tmem_ld32(t_o + 32 * q, o);
-                        tmem_wait_ld();
-                        reg_fence32(o);
+            for (int h = 0; h < 2; ++h) {
+                if constexpr (BN > 128) load_cols(h * kRegCols);
+                uint32_t pw[kHW];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        reg_fence32(o);
-                        tmem_st32(t_o + 32 * q, o);
+                for (int k = 0; k < kHW; ++k) {
+                    const int kk = kHW * h + k;                          // word index in the row
+                    const int sk = BN > 128 ? 2 * k : 2 * kk;            // its keys in s[]
+                    const uint64_t x2v = fma2(f2(__uint_as_float(s[sk]), __uint_as_float(s[sk + 1])), c2, negm);
+                    float e0, e1, p0, p1;
+                    f2_split(x2v, e0, e1);
+                    if (EMU > 0 && (kk % (EMU > 0 ? EMU : 1)) == EMU - 1) {
+                        exp2_poly2(e0, e1, p0, p1);
+                    } else {
+                        p0 = ex2_approx(e0);
+                        p1 = ex2_approx(e1);
                     }
+                    const uint32_t w = pack_bf16x2(p0, p1);
+                    const uint64_t pr = f2(p0, p1);
+                    // the bf16 halves of w added to fp32 sums directly (mixed-precision adds)
+                    if (k & 1) {
+                        la1 = add2(la1, pr);
+                        add_bf16x2_halves(hl1, hh1, w);
+                    } else {
+                        la0 = add2(la0, pr);
+                        add_bf16x2_halves(hl0, hh0, w);
+                    }
+                    pw[k] = w;
                 }
-                tmem_wait_st();
-                // keep the stored registers untouched until the stores completed
-                reg_fence32(p0);
-                reg_fence32(p1);
+                store_words<kHW>(t_p + kHW * h, pw);
+                tc_fence_before();
+                mbar_arrive(h == 0 ? bar_ph : bar_p);
             }
-            tc_fence_before();
-            mbar_arrive(bar_p);
-            float v0, v1, v2, v3;
+            float v0, v1;
             f2_split(add2(la0, la1), v0, v1);
-            f2_split(add2(ha0, ha1), v2, v3);
             l += v0 + v1;
-            lh += v2 + v3;
+            lh += (hl0 + hh0) + (hl1 + hh1);
         }
 
         // ------------------------------------------------------------ epilogue
@@ -325,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             wait_bar(bar_o_full + 8 * ti, 0, abort, p.status);
             tc_fence_after();
             // Q_i is dead (every product of issuer i has completed): stage O_i there
-            const uint32_t stage = base + C::kQOff + ti * C::kTileBytes;
+            const uint32_t stage = base + C::kQOff + ti * C::kQTileBytes;
             const uint32_t sw = static_cast<uint32_t>(r & 7);
             const float inv = lh > 0.f ? 1.f / lh : 0.f;
 #pragma unroll 1
@@ -335,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_ld();
                 reg_fence32(o);
                 // columns 32q .. 32q+31: box q/2, 16-byte chunks 4(q%2) .. 4(q%2)+3
-                const uint32_t rowaddr = stage + (q >> 1) * C::kBoxBytes + r * 128;
+                const uint32_t rowaddr = stage + (q >> 1) * C::kQBoxBytes + r * 128;
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                     const uint32_t ch = static_cast<uint32_t>(4 * (q & 1) + v);
@@ -356,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (quarter == 0 && lane == 0) {
 #pragma unroll
                 for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_store_3d(&tm_o, stage + bx * C::kBoxBytes, 64 * bx, q0, bh);
+                    tma_store_3d(&tm_o, stage + bx * C::kQBoxBytes, 64 * bx, q0, bh);
                 bulk_commit_group();
                 bulk_wait_group_read0();
             }
@@ -370,10 +409,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t slot_smem = base + C::kSlotOff;
             for (int i = 0; i < 2; ++i) {
                 if (kv_tiles(i) == 0) continue;
-                mbar_arrive_expect_tx(bar_q_full + 8 * i, C::kTileBytes);
+                mbar_arrive_expect_tx(bar_q_full + 8 * i, C::kQTileBytes);
 #pragma unroll
                 for (int bx = 0; bx < C::kBoxes; ++bx)
-                    tma_load_3d(base + C::kQOff + i * C::kTileBytes + bx * C::kBoxBytes, &tm_q, 64 * bx,
+                    tma_load_3d(base + C::kQOff + i * C::kQTileBytes + bx * C::kQBoxBytes, &tm_q, 64 * bx,
                                 256 * c + 128 * i, bh, bar_q_full + 8 * i, pol_q);
             }
             int ld = 0;
@@ -381,11 +420,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int t = 0; t < 2; ++t, ++ld) {
                     const int slot = ld % SLOTS, use = ld / SLOTS;
                     if (use > 0) wait_bar(bar_kv_empty + 8 * slot, (use - 1) & 1, abort, p.status);
-                    mbar_arrive_expect_tx(bar_kv_full + 8 * slot, C::kTileBytes);
+                    mbar_arrive_expect_tx(bar_kv_full + 8 * slot, C::kKVTileBytes);
 #pragma unroll
                     for (int bx = 0; bx < C::kBoxes; ++bx)
-                        tma_load_3d(slot_smem + slot * C::kTileBytes + bx * C::kBoxBytes, t ? &tm_v : &tm_k,
-                                    64 * bx, j * kBlockN, bh, bar_kv_full + 8 * slot, pol_kv);
+                        tma_load_3d(slot_smem + slot * C::kKVTileBytes + bx * C::kKVBoxBytes, t ? &tm_v : &tm_k,
+                                    64 * bx, j * BN, bh, bar_kv_full + 8 * slot, pol_kv);
                 }
             }
             // In an aborted CTA make sure no copy is still landing in shared
@@ -404,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const int n0 = kv_tiles(0), n1 = kv_tiles(1);
             const uint32_t slot_smem = base + C::kSlotOff;
-            const auto slot_addr = [&](int i) { return slot_smem + (i % SLOTS) * C::kTileBytes; };
+            const auto slot_addr = [&](int i) { return slot_smem + (i % SLOTS) * C::kKVTileBytes; };
             // Each ring load (K_j = load 2j, V_j = load 2j+1) is waited for once,
             // in load order, and released by one commit after its last use.
             int waited = -1;
@@ -417,32 +456,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Descriptors are built once; the start-address field (bits 0..13,
             // address >> 4) is advanced by plain integer adds, which never carry
             // out of the field for shared-memory addresses below 256 KiB.
-            constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false);
+            constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, BN, false);
             constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, true);
             const uint64_t desc_kmaj = smem_desc_sw128(0, 16, 1024);
             // V as the B operand is MN-major (d contiguous): 8-key groups 1024 bytes
-            // apart, 64-column halves of d one box (16 KiB) apart
-            const uint64_t desc_v = smem_desc_sw128(0, C::kBoxBytes, 1024);
+            // apart, 64-column halves of d one box (BN x 128 bytes) apart
+            const uint64_t desc_v = smem_desc_sw128(0, C::kKVBoxBytes, 1024);
             // S_ti(j) = Q_ti K_j^T into S_ti, then signal the softmax of tile ti
             const auto issue_s = [&](int ti, int j) {
-                const uint64_t a_q = desc_kmaj + ((base + C::kQOff + ti * C::kTileBytes) >> 4);
+                const uint64_t a_q = desc_kmaj + ((base + C::kQOff + ti * C::kQTileBytes) >> 4);
                 const uint64_t b_k = desc_kmaj + (slot_addr(2 * j) >> 4);
-                const uint32_t d_s = tmem + 128u * ti;
+                const uint32_t d_s = tmem + static_cast<uint32_t>(BN) * ti;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * C::kBoxBytes + (kk & 3) * 32) >> 4;
-                    mma_ss(d_s, a_q + off, b_k + off, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t a_off = ((kk >> 2) * C::kQBoxBytes + (kk & 3) * 32) >> 4;
+                    const uint32_t b_off = ((kk >> 2) * C::kKVBoxBytes + (kk & 3) * 32) >> 4;
+                    mma_ss(d_s, a_q + a_off, b_k + b_off, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar_s_full + 8 * ti);
             };
-            // O_ti += P_ti(j) V_j, P from TMEM (8 columns per 16 keys)
-            const auto issue_pv = [&](int ti, int j) {
+            // O_ti += P_ti(j) V_j for the keys of half h (BN/2 keys), P from TMEM
+            // (8 columns per 16 keys)
+            const auto issue_pv = [&](int ti, int j, int h) {
                 const uint64_t b_v = desc_v + (slot_addr(2 * j + 1) >> 4);
-                const uint32_t a_p = tmem + 128u * ti + C::kColP;
+                const uint32_t a_p = tmem + static_cast<uint32_t>(BN) * ti;
                 const uint32_t d_o = tmem + C::kColO + static_cast<uint32_t>(D) * ti;
 #pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk)
+                for (int k4 = 0; k4 < BN / 32; ++k4) {
+                    const int kk = (BN / 32) * h + k4;
                     mma_ts(d_o, a_p + kk * 8, b_v + kk * (2048 >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                }
             };
             // Order: S_0(0), S_1(0), then per key tile j the batch of tile 0
             // (O_0 += P_0(j) V_j, S_0(j+1)) and then that of tile 1.  The tensor
@@ -462,10 +505,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int ti = 0; ti < 2; ++ti) {
                     const int n_i = ti ? n1 : n0;
                     if (j >= n_i) continue;
-                    wait_bar(bar_p_full + 8 * ti, j & 1, abort, p.status);
+                    wait_bar(bar_p_half + 8 * ti, j & 1, abort, p.status);
                     tc_fence_after();
                     wait_kv(2 * j + 1);
-                    issue_pv(ti, j);
+                    issue_pv(ti, j, 0);
+                    wait_bar(bar_p_full + 8 * ti, j & 1, abort, p.status);
+                    tc_fence_after();
+                    issue_pv(ti, j, 1);
                     if (j + 1 < n_i) {
                         wait_kv(2 * j + 2);
                         issue_s(ti, j + 1);

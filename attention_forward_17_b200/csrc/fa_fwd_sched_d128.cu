@@ -5,8 +5,10 @@
 // ring's parity waits sound), plus the two persistent launches and the split-KV ping-pong kernel (P in shared
 // memory, which leaves room for a four-slot ring only) (one CTA per SM
 // walking several query tiles) for the default exponential split, and the
-// two-query-tile kernel (Q_0 and Q_1 take 64 KiB, so at most five slots; its
-// ring is sound at any depth) over the exponential split.  First entry =
+// two-query-tile kernel (Q_0 and Q_1 take 64 KiB, so at most five 128-row
+// slots; its ring is sound at any depth) over the exponential split and with
+// 64-row key tiles (two score and two output buffers of 2 x 192 + 2 x 128
+// columns would not fit TMEM, so no 192-row tiles at this head dimension).  First entry =
 // default.
 #include "fa_schedules.h"
 
@@ -20,6 +22,7 @@ const Schedule kD128[] = {
     make_pp_schedule<128, 4, 4>(), make_pp_schedule<128, 0, 4>(),
     make_2q_schedule<128, 4, 5>(), make_2q_schedule<128, 8, 5>(), make_2q_schedule<128, 2, 5>(),
     make_2q_schedule<128, 0, 5>(), make_2q_schedule<128, 4, 3>(),
+    make_2q_schedule<128, 4, 8, 64>(),
 };
 }  // namespace
 

@@ -1,7 +1,8 @@
 // Compiled schedules of the attention kernel for head dimension 64: the
 // exponential split (EMU) times the K/V ring depth (SLOTS, 16 KiB a slot),
 // plus the two persistent launches and the split-KV ping-pong kernel for the
-// default exponential split, and the two-query-tile kernel.  First entry =
+// default exponential split, and the two-query-tile kernel (key tiles of 64,
+// 128 and 192 rows: 2 x 192 + 2 x 64 = 512 TMEM columns).  First entry =
 // default.
 #include "fa_schedules.h"
 
@@ -16,6 +17,7 @@ const Schedule kD64[] = {
     make_pp_schedule<64, 0, 8>(),
     make_2q_schedule<64, 4, 8>(), make_2q_schedule<64, 2, 8>(), make_2q_schedule<64, 0, 8>(),
     make_2q_schedule<64, 4, 4>(),
+    make_2q_schedule<64, 4, 8, 64>(), make_2q_schedule<64, 4, 8, 192>(),
 };
 }  // namespace
 

@@ -1,6 +1,7 @@
 // Schedule table of the attention kernel: for each head dimension, masking
 // mode and sequence-length bucket (N <= n_max), the exponential split, the
-// K/V ring depth, the causal launch group, the launch form and the algorithm.  Written by
+// K/V ring depth, the causal launch group, the launch form, the algorithm and
+// the key-tile rows.  Written by
 // attention_forward_17_b200/schedule_search.py on NVIDIA B200 (2026-12-02).
 #pragma once
 
@@ -17,21 +18,22 @@ struct ScheduleTableEntry {
     int group;
     int persist;
     int alg;
+    int bn;
 };
 
 constexpr ScheduleTableEntry kScheduleTable[] = {
-    {128, 0, 2048, 4, 4, 1, 2, 0},
-    {128, 0, 8192, 4, 5, 1, 0, 0},
-    {128, 0, INT64_MAX, 4, 4, 1, 0, 1},
-    {128, 1, 2048, 4, 4, 16, 2, 0},
-    {128, 1, 8192, 4, 4, 4, 2, 0},
-    {128, 1, INT64_MAX, 4, 4, 16, 0, 1},
-    {64, 0, 2048, 4, 8, 1, 2, 0},
-    {64, 0, 8192, 4, 8, 1, 2, 0},
-    {64, 0, INT64_MAX, 4, 8, 1, 0, 0},
-    {64, 1, 2048, 4, 4, 1, 1, 0},
-    {64, 1, 8192, 4, 8, 16, 2, 0},
-    {64, 1, INT64_MAX, 4, 8, 16, 0, 1},
+    {128, 0, 2048, 4, 4, 1, 2, 0, 128},
+    {128, 0, 8192, 4, 5, 1, 0, 0, 128},
+    {128, 0, INT64_MAX, 4, 4, 1, 0, 1, 128},
+    {128, 1, 2048, 4, 4, 16, 2, 0, 128},
+    {128, 1, 8192, 4, 4, 4, 2, 0, 128},
+    {128, 1, INT64_MAX, 4, 4, 16, 0, 1, 128},
+    {64, 0, 2048, 4, 8, 1, 2, 0, 128},
+    {64, 0, 8192, 4, 8, 1, 2, 0, 128},
+    {64, 0, INT64_MAX, 4, 8, 1, 0, 0, 128},
+    {64, 1, 2048, 4, 4, 1, 1, 0, 128},
+    {64, 1, 8192, 4, 8, 16, 2, 0, 128},
+    {64, 1, INT64_MAX, 4, 8, 16, 0, 1, 128},
 };
 
 }  // namespace fa

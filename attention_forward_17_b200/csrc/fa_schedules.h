@@ -29,6 +29,7 @@ struct Schedule {
                        // (two softmax groups take alternate key tiles, merged at the end);
                        // 2: two query tiles per CTA, P over S in TMEM, one issuer per tile
     int smem_bytes;    // dynamic shared memory per CTA
+    int bn;            // rows of a key/value tile (128 except for algorithm 2)
     FwdLaunchFn launch[2];   // [causal]
     int (*setup)();          // shared-memory opt-in and register check, both modes
 };
@@ -73,23 +74,24 @@ constexpr Schedule make_pp_schedule() {
                     0,
                     1,
                     PPCfg<D, SLOTS>::kSmemBytes,
+                    128,
                     {&launch_pp<D, false, EMU, SLOTS>, &launch_pp<D, true, EMU, SLOTS>},
                     &setup_pp_both<D, EMU, SLOTS>};
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN>
 cudaError_t launch_2q(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                       const CUtensorMap& to, const FwdParams& p, unsigned grid, cudaStream_t stream) {
-    fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS>
-        <<<grid, kThreads, Q2Cfg<D, SLOTS>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+    fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN>
+        <<<grid, kThreads, Q2Cfg<D, SLOTS, BN>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN>
 int setup_2q_one() {
-    auto* k = fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS>;
+    auto* k = fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Q2Cfg<D, SLOTS>::kSmemBytes) != cudaSuccess)
+                             Q2Cfg<D, SLOTS, BN>::kSmemBytes) != cudaSuccess)
         return -6;
     cudaFuncAttributes attr;
     if (cudaFuncGetAttributes(&attr, k) != cudaSuccess) return -6;
@@ -97,23 +99,24 @@ int setup_2q_one() {
     return 0;
 }
 
-template <int D, int EMU, int SLOTS>
+template <int D, int EMU, int SLOTS, int BN>
 int setup_2q_both() {
-    const int rc = setup_2q_one<D, false, EMU, SLOTS>();
-    return rc ? rc : setup_2q_one<D, true, EMU, SLOTS>();
+    const int rc = setup_2q_one<D, false, EMU, SLOTS, BN>();
+    return rc ? rc : setup_2q_one<D, true, EMU, SLOTS, BN>();
 }
 
-// Two query tiles per CTA (fa_fwd_2q_kernel).
-template <int D, int EMU, int SLOTS>
+// Two query tiles per CTA (fa_fwd_2q_kernel), key tiles of BN rows.
+template <int D, int EMU, int SLOTS, int BN = 128>
 constexpr Schedule make_2q_schedule() {
     return Schedule{D,
                     EMU,
                     SLOTS,
                     0,
                     2,
-                    Q2Cfg<D, SLOTS>::kSmemBytes,
-                    {&launch_2q<D, false, EMU, SLOTS>, &launch_2q<D, true, EMU, SLOTS>},
-                    &setup_2q_both<D, EMU, SLOTS>};
+                    Q2Cfg<D, SLOTS, BN>::kSmemBytes,
+                    BN,
+                    {&launch_2q<D, false, EMU, SLOTS, BN>, &launch_2q<D, true, EMU, SLOTS, BN>},
+                    &setup_2q_both<D, EMU, SLOTS, BN>};
 }
 
 template <int D, bool CAUSAL, int EMU, int SLOTS, int PERSIST>
@@ -157,6 +160,7 @@ constexpr Schedule make_schedule() {
                     PERSIST,
                     0,
                     TileCfg<D, SLOTS>::kSmemBytes,
+                    128,
                     {&launch_schedule<D, false, EMU, SLOTS, PERSIST>,
                      &launch_schedule<D, true, EMU, SLOTS, PERSIST>},
                     &setup_both<D, EMU, SLOTS, PERSIST>};

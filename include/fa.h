@@ -127,9 +127,10 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
  *                     128-row query tiles per CTA sharing every key/value
  *                     tile, P kept over the scores in tensor memory, one
  *                     tensor-core issuing thread per query tile, O stored
- *                     through shared memory with TMA) and shared memory per CTA of
- *                     schedule `id`; FA_ERR_ARG for an unknown id.  Output
- *                     pointers may be NULL.
+ *                     through shared memory with TMA), shared memory per CTA
+ *                     and rows of a key/value tile (128, or 64 / 192 for some
+ *                     two-tile schedules) of schedule `id`; FA_ERR_ARG for an
+ *                     unknown id.  Output pointers may be NULL.
  * fa_fwd_pick_schedule - the schedule id and causal group fa_fwd uses for
  *                     (N, d, causal).  FA_ERR_NULL, FA_ERR_SHAPE (N < 0),
  *                     FA_ERR_HEADDIM.
@@ -143,7 +144,7 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
  */
 int fa_schedule_count(void);
 int fa_schedule_info(int id, int* d, int* emu_every, int* kv_slots, int* persistent,
-                     int* algorithm, int* smem_bytes);
+                     int* algorithm, int* smem_bytes, int* key_tile);
 int fa_fwd_pick_schedule(int64_t N, int64_t d, int causal, int* schedule_id, int* causal_group);
 int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
                     int64_t H, int64_t N, int64_t d, int causal, float scale, int schedule_id,

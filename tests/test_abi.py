@@ -35,7 +35,7 @@ def test_strerror_and_version():
         s = fa.strerror(code)
         assert isinstance(s, str) and s
     assert fa.strerror(12345) == "unknown status"
-    assert fa.version() == (1, 1)
+    assert fa.version() == (1, 2)
 
 
 def call(q=16, k=32, v=48, o=64, lse=80, B=1, H=1, N=128, d=64, causal=0, scale=0.125):
@@ -145,22 +145,26 @@ def test_schedule_registry():
     n = LIB.fa_schedule_count()
     assert n >= 2
     import ctypes
-    vals = [ctypes.c_int() for _ in range(6)]
+    vals = [ctypes.c_int() for _ in range(7)]
     seen = set()
     for i in range(n):
         assert LIB.fa_schedule_info(i, *[ctypes.byref(x) for x in vals]) == fa.FA_OK
-        d, emu, slots, persist, alg, smem = (x.value for x in vals)
+        d, emu, slots, persist, alg, smem, bn = (x.value for x in vals)
+        # key tiles of 128 rows, or 64 / 192 for the two-tile kernel where two
+        # score and two output buffers fit the 512 TMEM columns
+        assert bn == 128 or (alg == 2 and bn in (64, 192) and 2 * bn + 2 * d <= 512)
         assert d in (64, 128) and emu in (0, 2, 4, 8) and persist in (0, 1, 2)
         assert alg in (0, 1, 2) and 0 < smem <= 232448
         # the one-tile kernels need four slots for sound parity waits; the
         # two-tile kernel's issuers observe every load in order, so any depth >= 2
         assert slots >= (2 if alg == 2 else 4)
-        assert (d, emu, slots, persist, alg) not in seen
-        seen.add((d, emu, slots, persist, alg))
+        assert (d, emu, slots, persist, alg, bn) not in seen
+        seen.add((d, emu, slots, persist, alg, bn))
     assert any(k[3] == 1 for k in seen) and any(k[3] == 2 for k in seen)
     assert any(k[4] == 1 for k in seen) and any(k[4] == 2 and k[0] == d for k in seen for d in (64, 128))
-    assert LIB.fa_schedule_info(n, None, None, None, None, None, None) == fa.FA_ERR_ARG
-    assert LIB.fa_schedule_info(-1, None, None, None, None, None, None) == fa.FA_ERR_ARG
+    assert {(k[0], k[5]) for k in seen} >= {(128, 64), (128, 128), (64, 64), (64, 128), (64, 192)}
+    assert LIB.fa_schedule_info(n, None, None, None, None, None, None, None) == fa.FA_ERR_ARG
+    assert LIB.fa_schedule_info(-1, None, None, None, None, None, None, None) == fa.FA_ERR_ARG
     # the first schedule of each head dimension is the default
     assert fa.schedules()[0]["d"] == 128
 
@@ -212,13 +216,13 @@ def test_schedule_table_entries_are_compiled():
     import re
     import os
     path = os.path.join(os.path.dirname(fa.LIB_PATH), "csrc", "fa_schedule_table.h")
-    rows = re.findall(r"\{(\d+), (\d), (\w+), (\d), (\d), (\d+), (\d), (\d)\},", open(path).read())
+    rows = re.findall(r"\{(\d+), (\d), (\w+), (\d), (\d), (\d+), (\d), (\d), (\d+)\},", open(path).read())
     assert rows, "no table rows parsed"
-    compiled = {(s["d"], s["emu_every"], s["kv_slots"], s["persistent"], s["algorithm"])
+    compiled = {(s["d"], s["emu_every"], s["kv_slots"], s["persistent"], s["algorithm"], s["key_tile"])
                 for s in fa.schedules()}
     buckets = set()
-    for d, causal, n_max, emu, slots, group, persist, alg in rows:
-        key = (int(d), int(emu), int(slots), int(persist), int(alg))
+    for d, causal, n_max, emu, slots, group, persist, alg, bn in rows:
+        key = (int(d), int(emu), int(slots), int(persist), int(alg), int(bn))
         assert key in compiled, f"table row {key} is not a compiled schedule"
         assert int(group) >= 1
         buckets.add((int(d), int(causal), n_max))
@@ -233,8 +237,8 @@ def test_schedule_table_entries_are_compiled():
                 s = fa.schedules()[sid]
                 row = next(r for r in rows if int(r[0]) == d and int(r[1]) == int(causal)
                            and (r[2] == "INT64_MAX" or N <= int(r[2])))
-                assert (s["emu_every"], s["kv_slots"], s["persistent"], s["algorithm"]) == \
-                    (int(row[3]), int(row[4]), int(row[6]), int(row[7]))
+                assert (s["emu_every"], s["kv_slots"], s["persistent"], s["algorithm"], s["key_tile"]) == \
+                    (int(row[3]), int(row[4]), int(row[6]), int(row[7]), int(row[8]))
 
 
 def test_build_entry_does_not_need_the_library():
