@@ -11,12 +11,16 @@
 // Roles (384 threads):
 //   warps 0-3  softmax for query tile 0, warps 4-7 for query tile 1.  A thread
 //              owns one query row (TMEM lane = row, 32x32b accesses): a row's
-//              128 scores sit in one thread's registers, so row maxima and sums
-//              need no shuffles.
+//              scores of a key tile pass through one thread's registers, so
+//              row maxima and sums need no shuffles.
 //   warp 8     TMA producer: Q_0 and Q_1 once, then K_0, V_0, K_1, V_1, ...
 //              through one shared-memory ring (full / empty mbarriers).
-//   warp 9     MMA issuer (one thread): S_i = Q_i K_j^T and O_i += P_i V_j for
-//              both tiles, in a fixed alternating order.
+//   warp 9     MMA issuer: S_i = Q_i K_j^T and O_i += P_i V_j for both tiles,
+//              in a fixed alternating order.  The whole warp runs the issuing
+//              loop and one elected lane issues each instruction, which keeps
+//              the descriptor arithmetic warp-uniform (issuing from a lone lane
+//              in a divergent branch cost 65-85 cycles per product, more than
+//              the 64 the tensor core needs for one).
 //   warp 10    allocates and frees TMEM.
 //
 // Key tiles are BN rows (BN = 64, 128 or 192, a template parameter; the tile
@@ -27,9 +31,9 @@
 // P_i straight from TMEM (the tensor core's TMEM-A form), so P never touches
 // shared memory.
 //
-// Why a single issuing thread: tcgen05 operations of one thread complete in
-// issue order, and an mbarrier commit fires once every earlier operation of
-// that thread has completed.  The issuer issues
+// Why a single issuing thread (the elected lane): tcgen05 operations of one
+// thread complete in issue order, and an mbarrier commit fires once every
+// earlier operation of that thread has completed.  The issuer issues
 //     S_0(0), S_1(0), [PV_0(0), S_0(1)], [PV_1(0), S_1(1)], [PV_0(1), S_0(2)], ...
 // so (a) S_i(j+1), which overwrites P_i(j), is issued after the product that
 // reads P_i(j); (b) when the softmax sees S_i(j) complete, PV_i(j-1) has
@@ -40,10 +44,10 @@
 // groups received their scores together and competed for the exponential
 // unit while the tensor core idled: 850-890 TFLOP/s against 1050-1100 for the
 // one-tile kernels at B=1, H=32, N=16384, d=128).
-// The lazy O rescale (a row's maximum grew by more than 2^8) is therefore done
-// in place by the softmax thread that owns the row, between its P store and
-// its release of P, with no wait on the tensor core: the rescale is off the
-// tensor pipe's critical path and costs only the TMEM round trip of that row.
+// The lazy O rescale (a row's maximum grew by more than 2^16) is therefore done
+// in place by the softmax thread that owns the row, before it releases P, with
+// no wait on the tensor core: the rescale costs only the TMEM round trip of
+// that row (no correction warps and no barrier round trip are needed).
 // While softmax group 0 works on S_0(j), the tensor core runs tile 1's
 // products, and the other way round, so the exponentials of one tile overlap
 // the matrix products of the other.
@@ -56,8 +60,8 @@
 //
 // Causal mask: query tile i of pair c needs the key tiles that hold keys
 // 0 .. 256c + 128i + 127; the ring carries those of tile 1 and the last ones
-// only feed tile 1.  The
-// issuer waits for every ring load exactly once, in load order, which keeps
+// only feed tile 1.  The issuer waits for every ring load exactly once, in
+// load order, which keeps
 // every parity wait on the ring sound for any depth (it waits for load L only
 // after observing load L-1), and releases each load by one commit after its
 // last use.
@@ -126,6 +130,13 @@ __device__ __forceinline__ void store_words(uint32_t taddr, uint32_t (&w)[N]) {
     for (int q = 0; q < N / 32; ++q) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&w[32 * q]));
     if constexpr (N % 32) reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&w[N - 16]));
 }
+
+// Lazy rescale threshold (log2 units): O and the sums are rescaled only when a
+// row's maximum grows by more than this, so P is bounded by 2^16 (exact range
+// for bf16 and fp32; the sums stay below 2^16 times the number of keys).  On
+// q, k ~ N(0, 3^2) scores a threshold of 16 instead of 8 shortened the step
+// of the two tiles by a tenth (fewer rescales).
+constexpr float kRescaleTau = 16.0f;
 
 constexpr int kQ2IssuerWarp = 9;       // issues every tcgen05.mma of the CTA
 constexpr int kQ2AllocWarp = 10;
@@ -279,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float mn =
                 fmaxf(max3f(x[0], x[1], x[2]), max3f(x[3], x[4], fmaxf(x[5], max3f(x[6], x[7], x[7])))) * cl;
-            const bool grow = mn > m + 8.0f;
+            const bool grow = mn > m + kRescaleTau;
             float alpha = 1.f;
             if (grow) {
                 alpha = ex2_approx(m - mn);
@@ -440,7 +451,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kQ2IssuerWarp) {
         regs_decrease<kRegsOther>();
         // ============================================================ MMA issuer (both tiles)
-        if (lane == 0) {
+        // The whole warp runs the issuing loop (converged, so the descriptor
+        // arithmetic stays warp-uniform); one elected lane issues each product
+        // and commit.
+        {
             const int n0 = kv_tiles(0), n1 = kv_tiles(1);
             const uint32_t slot_smem = base + C::kSlotOff;
             const auto slot_addr = [&](int i) { return slot_smem + (i % SLOTS) * C::kKVTileBytes; };
@@ -471,9 +485,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t a_off = ((kk >> 2) * C::kQBoxBytes + (kk & 3) * 32) >> 4;
                     const uint32_t b_off = ((kk >> 2) * C::kKVBoxBytes + (kk & 3) * 32) >> 4;
-                    mma_ss(d_s, a_q + a_off, b_k + b_off, idesc_s, kk > 0 ? 1u : 0u);
+                    mma_ss_elect(d_s, a_q + a_off, b_k + b_off, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(bar_s_full + 8 * ti);
+                mma_commit_elect(bar_s_full + 8 * ti);
             };
             // O_ti += P_ti(j) V_j for the keys of half h (BN/2 keys), P from TMEM
             // (8 columns per 16 keys)
@@ -484,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int k4 = 0; k4 < BN / 32; ++k4) {
                     const int kk = (BN / 32) * h + k4;
-                    mma_ts(d_o, a_p + kk * 8, b_v + kk * (2048 >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts_elect(d_o, a_p + kk * 8, b_v + kk * (2048 >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 }
             };
             // Order: S_0(0), S_1(0), then per key tile j the batch of tile 0
@@ -500,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 issue_s(1, 0);
             }
-            mma_commit(bar_kv_empty);                    // K_0 (slot 0)
+            mma_commit_elect(bar_kv_empty);                    // K_0 (slot 0)
             for (int j = 0; j < n_kv; ++j) {
                 for (int ti = 0; ti < 2; ++ti) {
                     const int n_i = ti ? n1 : n0;
@@ -516,11 +530,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         wait_kv(2 * j + 2);
                         issue_s(ti, j + 1);
                     } else {
-                        mma_commit(bar_o_full + 8 * ti);
+                        mma_commit_elect(bar_o_full + 8 * ti);
                     }
                 }
-                mma_commit(bar_kv_empty + 8 * ((2 * j + 1) % SLOTS));            // V_j
-                if (j + 1 < n_kv) mma_commit(bar_kv_empty + 8 * ((2 * j + 2) % SLOTS));   // K_{j+1}
+                mma_commit_elect(bar_kv_empty + 8 * ((2 * j + 1) % SLOTS));            // V_j
+                if (j + 1 < n_kv) mma_commit_elect(bar_kv_empty + 8 * ((2 * j + 2) % SLOTS));   // K_{j+1}
             }
             // every product has completed before TMEM is released
             wait_bar(bar_o_full, 0, abort, p.status);

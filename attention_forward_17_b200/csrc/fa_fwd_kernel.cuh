@@ -146,17 +146,12 @@ __device__ __forceinline__ int load_index_v(int t, int n) {
 // Polls the mbarrier phase until it completes or `limit_ns` (globaltimer)
 // passes; on time-out marks the CTA aborted and records FA_ERR_TIMEOUT.  Once
 // aborted, further waits give up after `limit_abort_ns`.
-#ifndef FA_WAIT_SUSPEND_NS
-#define FA_WAIT_SUSPEND_NS 0
-#endif
 __device__ __forceinline__ void wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort,
                                           int* status, uint64_t limit_ns, uint64_t limit_abort_ns) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (FA_WAIT_SUSPEND_NS > 0 ? mbar_try_wait_sleep(bar, parity, FA_WAIT_SUSPEND_NS)
-                                   : mbar_try_wait(bar, parity))
-            return;
-        if (FA_WAIT_SUSPEND_NS > 0 || (it & 31u) == 0) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((it & 31u) == 0) {
             const uint64_t limit = *abort ? limit_abort_ns : limit_ns;
             if (global_timer_ns() - t0 > limit) {
                 if (!*abort) {

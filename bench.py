@@ -70,14 +70,18 @@ def load_peaks():
         return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
 
 
+KERNEL_FAMILY = {0: "fa_fwd_kernel", 1: "fa_fwd_pp_kernel", 2: "fa_fwd_2q_kernel"}
+
+
 def measured_traffic(workload, algorithm=0):
     """DRAM bytes per non-causal launch from the committed ncu summary of the
     kernel family the headline runs (algorithm 0: fa_fwd_kernel, 1: the split-KV
-    ping-pong kernel), or None when that kernel's source changed since the
-    counters were taken (or the summary does not cover this workload)."""
+    ping-pong kernel, 2: the two-query-tile kernel), or None when that kernel's
+    source changed since the counters were taken (or the summary does not cover
+    this workload)."""
     if workload != DEFAULT_WORKLOAD:
         return None, None
-    name = "fa_fwd_pp_kernel" if algorithm == 1 else "fa_fwd_kernel"
+    name = KERNEL_FAMILY[algorithm]
     prof = os.path.join(ROOT, "profiles", f"{name}_b1_h64_n4096_d128_ncu.md")
     src = os.path.join(ROOT, "attention_forward_17_b200", "csrc", f"{name}.cuh")
     try:
@@ -250,7 +254,7 @@ def schedule_of(N, d, causal, schedule=None, causal_group=None):
     grp = grp if causal_group is None else causal_group
     s = fa.schedules()[sid]
     return {"id": sid, "exp_poly_every": s["emu_every"], "kv_slots": s["kv_slots"],
-            "persistent": s["persistent"], "algorithm": s["algorithm"],
+            "persistent": s["persistent"], "algorithm": s["algorithm"], "key_tile": s["key_tile"],
             "causal_group": grp if (causal and s["persistent"] != 1) else None}
 
 
@@ -364,7 +368,7 @@ def run_ours(args, cfg):
     dominant = max(modes, key=lambda c: launch_ms[c])
     sch_dom = schedule_of(N, d, dominant, args.schedule, args.causal_group)
     traffic, traffic_src = measured_traffic(args.workload, sch_dom["algorithm"])
-    kname = "fa_fwd_pp_kernel" if sch_dom["algorithm"] == 1 else "fa_fwd_kernel"
+    kname = KERNEL_FAMILY[sch_dom["algorithm"]]
     roofline = {"bound": "tensor", "kernel": f"{kname} d={d} {'causal' if dominant else 'non-causal'} "
                                              f"schedule {sch_dom['id']}",
                 "achieved": ach[dominant], "peak": peaks["bf16"], "unit": "TFLOP/s",

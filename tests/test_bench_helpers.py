@@ -32,12 +32,15 @@ def test_profile_traffic_is_gated_by_the_source_hash(tmp_path, monkeypatch):
 def test_headline_traffic_follows_the_kernel_family():
     # each kernel family reads its own summary; the figure is reported while the
     # summary's source hash matches the kernel, and withheld (with the reason) after
-    for alg, name in ((0, "fa_fwd_kernel"), (1, "fa_fwd_pp_kernel")):
+    for alg, name in ((0, "fa_fwd_kernel"), (1, "fa_fwd_pp_kernel"), (2, "fa_fwd_2q_kernel")):
         val, why = bench.measured_traffic(bench.DEFAULT_WORKLOAD, alg)
+        prof = os.path.join(bench.ROOT, "profiles", f"{name}_b1_h64_n4096_d128_ncu.md")
         if val is not None:
             assert val > 0 and name in why
-        else:
+        elif os.path.exists(prof):
             assert why == "kernel changed since the ncu capture"
+        else:
+            assert why is None          # no capture of this kernel family committed
     # other workloads are not covered by the profiling capture
     assert bench.measured_traffic("b2_h16_n4096_d128", 0) == (None, None)
 
