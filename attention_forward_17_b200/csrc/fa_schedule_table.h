@@ -2,7 +2,7 @@
 // mode and sequence-length bucket (N <= n_max), the exponential split, the
 // K/V ring depth, the causal launch group, the launch form, the algorithm and
 // the key-tile rows.  Written by
-// attention_forward_17_b200/schedule_search.py on NVIDIA B200 (2026-12-02).
+// attention_forward_17_b200/schedule_search.py on NVIDIA B200 (2026-12-03).
 #pragma once
 
 #include <cstdint>
@@ -22,18 +22,18 @@ struct ScheduleTableEntry {
 };
 
 constexpr ScheduleTableEntry kScheduleTable[] = {
-    {128, 0, 2048, 4, 4, 1, 2, 0, 128},
-    {128, 0, 8192, 4, 5, 1, 0, 0, 128},
-    {128, 0, INT64_MAX, 4, 4, 1, 0, 1, 128},
-    {128, 1, 2048, 4, 4, 16, 2, 0, 128},
-    {128, 1, 8192, 4, 4, 4, 2, 0, 128},
-    {128, 1, INT64_MAX, 4, 4, 16, 0, 1, 128},
-    {64, 0, 2048, 4, 8, 1, 2, 0, 128},
-    {64, 0, 8192, 4, 8, 1, 2, 0, 128},
-    {64, 0, INT64_MAX, 4, 8, 1, 0, 0, 128},
+    {128, 0, 2048, 4, 5, 1, 0, 2, 128},
+    {128, 0, 8192, 0, 5, 1, 0, 2, 128},
+    {128, 0, INT64_MAX, 4, 5, 1, 0, 2, 128},
+    {128, 1, 2048, 4, 5, 16, 0, 2, 128},
+    {128, 1, 8192, 0, 5, 16, 0, 2, 128},
+    {128, 1, INT64_MAX, 8, 5, 4, 0, 2, 128},
+    {64, 0, 2048, 4, 4, 1, 0, 2, 128},
+    {64, 0, 8192, 4, 8, 1, 0, 2, 128},
+    {64, 0, INT64_MAX, 4, 4, 1, 0, 2, 128},
     {64, 1, 2048, 4, 4, 1, 1, 0, 128},
-    {64, 1, 8192, 4, 8, 16, 2, 0, 128},
-    {64, 1, INT64_MAX, 4, 8, 16, 0, 1, 128},
+    {64, 1, 8192, 4, 8, 16, 0, 2, 128},
+    {64, 1, INT64_MAX, 4, 8, 16, 0, 2, 128},
 };
 
 }  // namespace fa

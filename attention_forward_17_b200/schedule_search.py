@@ -25,7 +25,9 @@ timed in three rounds that start at different candidates and keep their best
 round, so the drift of the clock as the GPU approaches its power cap does not
 favour whichever candidate is timed first.  Each candidate's output is first
 checked against the default schedule's (the parity tests pin every schedule
-to the fp64 oracle).  A candidate replaces the default only if it is more than
+to the fp64 oracle; two outputs that each meet the oracle's bars can differ by
+up to twice them, which is the bound used here).  A candidate replaces the
+default only if it is more than
 1 % faster.  Buckets and their timed problem (N B H = 16 * 16384 query rows):
 
     N <= 2048   N = 1024,  B = 16, H = 16, q, k ~ N(0, 1)
@@ -117,7 +119,11 @@ def search(log=print):
                     do = (o.float() - ref_o.float()).abs().max().item()
                     dl = (lse - ref_l).abs().max().item()
                     rel = ((o.float() - ref_o.float()).norm() / ref_o.float().norm()).item()
-                    ok = do <= 2e-2 and dl <= 1e-3 and rel <= 1e-2 and bool(torch.isfinite(o.float()).all())
+                    # both outputs are held to the fp64 oracle's bars (2e-2 max-abs and
+                    # 1e-2 rel-L2 on O, 1e-3 on LSE) by the parity tests; two outputs
+                    # within those bars can differ by up to twice them (one bf16 step of
+                    # an |O| >= 4 value is already 2^-5), so twice the bars here
+                    ok = do <= 4e-2 and dl <= 2e-3 and rel <= 2e-2 and bool(torch.isfinite(o.float()).all())
                     valid.append((ok, do, dl))
                 best = [(0.0, None)] * len(cand)
                 for rep in range(REPS):
@@ -204,7 +210,8 @@ def write_report(rows, table, device_name, path, top=6):
            f"(rotated order) of {WARMUP} warm-up + {ITERS} timed launches (CUDA events), the way the "
            "benchmark times the headline; MHz = median SM clock sampled (NVML, 10 ms) during that "
            "round's timed launches; per GHz = TFLOP/s / (MHz / 1000); reasons = clock-event reasons "
-           "seen. `ok` = output within the parity tolerances of the default schedule's. alg: 0 one "
+           "seen. `ok` = output within twice the oracle's parity bars of the default schedule's (each "
+           "is held to the oracle's bars by the parity tests). alg: 0 one "
            "query tile per CTA, 1 split-KV ping-pong, 2 two query tiles per CTA; launch: 0 one CTA "
            "per tile, 1 static persistent, 2 cluster launch control.", ""]
     keys = []
