@@ -234,7 +234,7 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
     p.rescale_stats = rescale_stats;
     int64_t grid = BH * p.n_qtile;
     if (grid > 0x7fffffffLL) return FA_ERR_SHAPE;
-    if (sch->alg == 2) {
+    if (sch->alg >= 2) {
         // two query tiles per CTA
         grid = BH * ((p.n_qtile + 1) / 2);
     } else if (sch->persist == 1) {

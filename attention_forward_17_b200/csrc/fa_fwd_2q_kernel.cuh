@@ -73,11 +73,13 @@
 
 namespace fa {
 
-template <int D, int SLOTS, int BN>
+template <int D, int SLOTS, int BN, bool DB, bool LT>
 struct Q2Cfg {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
     static_assert(BN == 64 || BN == 128 || BN == 192, "key tile of 64, 128 or 192 rows");
-    static_assert(SLOTS >= 2, "K/V ring depth");
+    // with double-buffered scores the issuer needs K_{j+2} while V_j is still
+    // unreleased: four loads in flight
+    static_assert(SLOTS >= (DB ? 4 : 2), "K/V ring depth");
     static constexpr int kQTileBytes = 128 * D * 2;         // one 128-row tile of Q (or O)
     static constexpr int kKVTileBytes = BN * D * 2;         // one BN-row tile of K or V
     static constexpr int kBoxes = D / 64;                   // 64-column (128-byte) TMA boxes
@@ -86,15 +88,27 @@ struct Q2Cfg {
     static constexpr int kSlots = SLOTS;
     static constexpr int kQOff = 0;                         // Q_0, then Q_1 (O staging at the end)
     static constexpr int kSlotOff = 2 * kQTileBytes;
-    static constexpr int kBarOff = kSlotOff + SLOTS * kKVTileBytes;
+    // LT: a BN-row tile of bf16 ones after the ring; the P.V product reads it as
+    // 16 extra columns of V, so O gains 16 columns that each accumulate the sum
+    // of the bf16 weights (l^) on the tensor core
+    static_assert(!LT || D == 64, "the ones tile is addressed as V's second 64-column chunk");
+    static constexpr int kOnesOff = kSlotOff + SLOTS * kKVTileBytes;
+    static constexpr int kOnesBytes = LT ? BN * 128 : 0;
+    static constexpr int kBarOff = kOnesOff + kOnesBytes;
+    static constexpr int kDO = D + (LT ? 16 : 0);           // columns of one O buffer
     static constexpr int kSmemBytes = 1024 /* alignment slack */ + kBarOff + 512;
-    // TMEM: S_0 [0,BN), S_1 [BN,2BN), O_0 [2BN,2BN+D), O_1 [2BN+D,2BN+2D); P_i
-    // (bf16 pairs, BN/2 columns) over the first columns of S_i
-    static constexpr uint32_t kColO = 2 * BN;
+    // TMEM: the score buffers of tile 0, then those of tile 1 (one each, or two
+    // each with DB), then O_0 and O_1 (D columns each); P (bf16 pairs, BN/2
+    // columns) over the first columns of the score buffer it was computed from
+    static constexpr int kSBufs = DB ? 2 : 1;
+    __host__ __device__ static constexpr uint32_t col_s(int ti, int b) {
+        return static_cast<uint32_t>((ti * kSBufs + b) * BN);
+    }
+    static constexpr uint32_t kColO = 2 * kSBufs * BN;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr int kHalfWords = BN / 4;               // P words released at a time
     static_assert(kSmemBytes <= 232448, "shared memory per CTA (227 KiB)");
-    static_assert(kColO + 2 * D <= kTmemCols, "two score and two output buffers in TMEM");
+    static_assert(kColO + 2 * kDO <= kTmemCols, "score and output buffers in TMEM");
     static_assert(kKVBoxBytes % 1024 == 0, "slots on 1024-byte boundaries (128-byte swizzle)");
 };
 
@@ -103,9 +117,15 @@ struct alignas(8) Q2Barriers {
     uint64_t kv_full[kSlots];
     uint64_t kv_empty[kSlots];     // released by one commit after the load's last use
     uint64_t q_full[2];
-    uint64_t s_full[2];            // S_i(j) computed (and PV_i(j-1) completed)
-    uint64_t p_half[2];            // first half of P_i(j)'s keys in TMEM, O_i rescaled (128 arrivals)
-    uint64_t p_full[2];            // second half of P_i(j)'s keys in TMEM (128 arrivals)
+    uint64_t s_full[4];            // [2i + b]: S_i(j) computed into score buffer b
+    // [2i + b]: the first / second half of P_i(j)'s keys in score buffer b (O_i
+    // rescaled before the first), 128 arrivals.  One pair per score buffer:
+    // with two buffers the softmax can release P_i(j+1) before the issuer has
+    // waited for P_i(j), and a single barrier would then be two phases ahead
+    // of that parity wait.
+    uint64_t p_half[4];
+    uint64_t p_full[4];
+    uint64_t pv_done[2];           // O_i += P_i(j) V_j completed (double-buffered scores)
     uint64_t o_full[2];            // every product of tile i completed
     uint32_t tmem_base;
     volatile uint32_t abort;
@@ -160,12 +180,12 @@ __device__ __forceinline__ void map_pair(const FwdParams& p, int n_pair, int id,
     }
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS, int BN>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                      const FwdParams p) {
-    using C = Q2Cfg<D, SLOTS, BN>;
+    using C = Q2Cfg<D, SLOTS, BN, DB, LT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -193,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_s_full = smem_u32(&bars->s_full[0]);
     const uint32_t bar_p_half = smem_u32(&bars->p_half[0]);
     const uint32_t bar_p_full = smem_u32(&bars->p_full[0]);
+    const uint32_t bar_pv_done = smem_u32(&bars->pv_done[0]);
     const uint32_t bar_o_full = smem_u32(&bars->o_full[0]);
     volatile uint32_t* abort = &bars->abort;
 
@@ -201,11 +222,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar_kv_full + 8 * s, 1);
             mbar_init(bar_kv_empty + 8 * s, 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(bar_q_full + 8 * i, 1);
+        for (int i = 0; i < 4; ++i) {
             mbar_init(bar_s_full + 8 * i, 1);
             mbar_init(bar_p_half + 8 * i, 128);
             mbar_init(bar_p_full + 8 * i, 128);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_q_full + 8 * i, 1);
+            mbar_init(bar_pv_done + 8 * i, 1);
             mbar_init(bar_o_full + 8 * i, 1);
         }
         bars->abort = 0u;
@@ -214,6 +238,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kQ2AllocWarp) {
         tmem_alloc(smem_u32(&bars->tmem_base), C::kTmemCols);
         tmem_relinquish();
+    }
+    if constexpr (LT) {
+        // the ones tile (bf16 1.0 everywhere, so its swizzled layout needs no care),
+        // written by the 256 softmax threads and made visible to the tensor core
+        if (warp < 8) {
+            const uint32_t ones = base + C::kOnesOff;
+#pragma unroll 1
+            for (int i = threadIdx.x; i < C::kOnesBytes / 16; i += 256)
+                st_shared_v4(ones + 16 * i, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+            fence_proxy_async_smem();
+        }
     }
     if (warp == kProducerWarp && lane == 0) {
         tma_prefetch_desc(&tm_q);
@@ -236,18 +271,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = q0 + r;
         const int n_i = kv_tiles(ti);
         const uint32_t lane_w = static_cast<uint32_t>(32 * quarter) << 16;
-        const uint32_t t_s = tmem + lane_w + static_cast<uint32_t>(BN) * ti;
-        const uint32_t t_p = t_s;
-        const uint32_t t_o = tmem + lane_w + C::kColO + static_cast<uint32_t>(D) * ti;
+        const uint32_t t_s0 = tmem + lane_w + C::col_s(ti, 0);
+        const uint32_t t_o = tmem + lane_w + C::kColO + static_cast<uint32_t>(C::kDO) * ti;
         const float cl = p.scale_log2;
         const uint64_t c2 = f2(cl, cl);
-        const uint32_t bar_s = bar_s_full + 8 * ti, bar_p = bar_p_full + 8 * ti;
-        const uint32_t bar_ph = bar_p_half + 8 * ti;
+
 
         float m = -INFINITY;                      // running max of c*s (stale by < 8)
         float l = 0.f, lh = 0.f;                  // sums of the weights: fp32, and bf16-rounded
         for (int j = 0; j < n_i; ++j) {
-            wait_bar(bar_s, j & 1, abort, p.status);
+            // score buffer of this step: with DB, S_i(j) sits in buffer j % 2
+            const int sb = DB ? (j & 1) : 0;
+            const uint32_t t_s = t_s0 + sb * BN, t_p = t_s;
+            wait_bar(bar_s_full + 8 * (2 * ti + sb), (DB ? (j >> 1) : j) & 1, abort, p.status);
             tc_fence_after();
             const bool masked =
                 (j * BN + BN > p.N) || (CAUSAL && j * BN + BN - 1 > q0);
@@ -298,11 +334,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l *= alpha;
                 lh *= alpha;
             }
-            // Lazy rescale of this row of O_i (O_i holds the products of steps
-            // < j, all completed: S_i(j) was issued after PV_i(j-1)).  The stores
+            // Lazy rescale of this row of O_i.  O_i holds the products of steps
+            // < j: with one score buffer they have all completed (S_i(j) was
+            // issued after PV_i(j-1)); with two, S_i(j) was issued before
+            // PV_i(j-1), so the rescale first waits for that product.  The stores
             // complete before the first release of P below (tcgen05.wait::st).
             const bool need = grow && j > 0;
             if (__any_sync(0xffffffffu, need)) {
+                if constexpr (DB) {
+                    wait_bar(bar_pv_done + 8 * ti, (j - 1) & 1, abort, p.status);
+                    tc_fence_after();
+                }
                 const unsigned rows = __popc(__ballot_sync(0xffffffffu, need));
                 if (p.rescale_stats && lane == 0) {
                     atomicAdd(p.rescale_stats, 1ull);
@@ -319,6 +361,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                     reg_fence32(o);
                     tmem_st32(t_o + 32 * q, o);
+                }
+                if constexpr (LT) {
+                    // the l^ columns of O
+                    uint32_t o[16];
+                    tmem_ld32x16(t_o + D, o);
+                    tmem_wait_ld();
+                    reg_fence16(o);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    reg_fence16(o);
+                    tmem_st16(t_o + D, o);
                 }
             }
             const float u = (m == -INFINITY) ? 0.f : m;
@@ -350,19 +403,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const uint32_t w = pack_bf16x2(p0, p1);
                     const uint64_t pr = f2(p0, p1);
-                    // the bf16 halves of w added to fp32 sums directly (mixed-precision adds)
+                    // the bf16 halves of w added to fp32 sums directly (mixed-precision
+                    // adds), unless the tensor core sums them (LT)
                     if (k & 1) {
                         la1 = add2(la1, pr);
-                        add_bf16x2_halves(hl1, hh1, w);
+                        if constexpr (!LT) add_bf16x2_halves(hl1, hh1, w);
                     } else {
                         la0 = add2(la0, pr);
-                        add_bf16x2_halves(hl0, hh0, w);
+                        if constexpr (!LT) add_bf16x2_halves(hl0, hh0, w);
                     }
                     pw[k] = w;
                 }
                 store_words<kHW>(t_p + kHW * h, pw);
                 tc_fence_before();
-                mbar_arrive(h == 0 ? bar_ph : bar_p);
+                mbar_arrive((h == 0 ? bar_p_half : bar_p_full) + 8 * (2 * ti + sb));
             }
             float v0, v1;
             f2_split(add2(la0, la1), v0, v1);
@@ -377,6 +431,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Q_i is dead (every product of issuer i has completed): stage O_i there
             const uint32_t stage = base + C::kQOff + ti * C::kQTileBytes;
             const uint32_t sw = static_cast<uint32_t>(r & 7);
+            if constexpr (LT) {
+                // l^ accumulated by the tensor core in the extra columns of O
+                uint32_t t[16];
+                tmem_ld32x16(t_o + D, t);
+                tmem_wait_ld();
+                reg_fence16(t);
+                lh = __uint_as_float(t[0]);
+            }
             const float inv = lh > 0.f ? 1.f / lh : 0.f;
 #pragma unroll 1
             for (int q = 0; q < D / 32; ++q) {
@@ -459,82 +521,102 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t slot_smem = base + C::kSlotOff;
             const auto slot_addr = [&](int i) { return slot_smem + (i % SLOTS) * C::kKVTileBytes; };
             // Each ring load (K_j = load 2j, V_j = load 2j+1) is waited for once,
-            // in load order, and released by one commit after its last use.
+            // in load order (waiting for load i first waits for every earlier
+            // one), and released by one commit after its last use.
             int waited = -1;
             const auto wait_kv = [&](int i) {
                 if (i <= waited) return;
-                wait_bar(bar_kv_full + 8 * (i % SLOTS), (i / SLOTS) & 1, abort, p.status);
+                while (waited < i) {
+                    ++waited;
+                    wait_bar(bar_kv_full + 8 * (waited % SLOTS), (waited / SLOTS) & 1, abort, p.status);
+                }
                 tc_fence_after();
-                waited = i;
             };
             // Descriptors are built once; the start-address field (bits 0..13,
             // address >> 4) is advanced by plain integer adds, which never carry
             // out of the field for shared-memory addresses below 256 KiB.
             constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, BN, false);
-            constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, true);
+            constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, C::kDO, true);
             const uint64_t desc_kmaj = smem_desc_sw128(0, 16, 1024);
             // V as the B operand is MN-major (d contiguous): 8-key groups 1024 bytes
             // apart, 64-column halves of d one box (BN x 128 bytes) apart
             const uint64_t desc_v = smem_desc_sw128(0, C::kKVBoxBytes, 1024);
-            // S_ti(j) = Q_ti K_j^T into S_ti, then signal the softmax of tile ti
+            // S_ti(j) = Q_ti K_j^T into its score buffer, then signal the softmax
+            // of tile ti
             const auto issue_s = [&](int ti, int j) {
+                const int sb = DB ? (j & 1) : 0;
                 const uint64_t a_q = desc_kmaj + ((base + C::kQOff + ti * C::kQTileBytes) >> 4);
                 const uint64_t b_k = desc_kmaj + (slot_addr(2 * j) >> 4);
-                const uint32_t d_s = tmem + static_cast<uint32_t>(BN) * ti;
+                const uint32_t d_s = tmem + C::col_s(ti, sb);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t a_off = ((kk >> 2) * C::kQBoxBytes + (kk & 3) * 32) >> 4;
                     const uint32_t b_off = ((kk >> 2) * C::kKVBoxBytes + (kk & 3) * 32) >> 4;
                     mma_ss_elect(d_s, a_q + a_off, b_k + b_off, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                mma_commit_elect(bar_s_full + 8 * ti);
+                mma_commit_elect(bar_s_full + 8 * (2 * ti + sb));
             };
             // O_ti += P_ti(j) V_j for the keys of half h (BN/2 keys), P from TMEM
             // (8 columns per 16 keys)
             const auto issue_pv = [&](int ti, int j, int h) {
-                const uint64_t b_v = desc_v + (slot_addr(2 * j + 1) >> 4);
-                const uint32_t a_p = tmem + static_cast<uint32_t>(BN) * ti;
-                const uint32_t d_o = tmem + C::kColO + static_cast<uint32_t>(D) * ti;
+                const uint32_t v_addr = slot_addr(2 * j + 1);
+                // LT: V's second 64-column chunk (one chunk stride, LBO, further on)
+                // is the ones tile, which follows the ring
+                const uint64_t b_v =
+                    (LT ? smem_desc_sw128(0, base + C::kOnesOff - v_addr, 1024) : desc_v) + (v_addr >> 4);
+                const uint32_t a_p = tmem + C::col_s(ti, DB ? (j & 1) : 0);
+                const uint32_t d_o = tmem + C::kColO + static_cast<uint32_t>(C::kDO) * ti;
 #pragma unroll
                 for (int k4 = 0; k4 < BN / 32; ++k4) {
                     const int kk = (BN / 32) * h + k4;
                     mma_ts_elect(d_o, a_p + kk * 8, b_v + kk * (2048 >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 }
             };
-            // Order: S_0(0), S_1(0), then per key tile j the batch of tile 0
-            // (O_0 += P_0(j) V_j, S_0(j+1)) and then that of tile 1.  The tensor
-            // core runs one tile's batch while the other tile's softmax works, and
-            // the two softmax groups stay half a step apart.
-            wait_bar(bar_q_full, 0, abort, p.status);
-            tc_fence_after();
-            wait_kv(0);
-            issue_s(0, 0);
-            if (n1 > 0) {
-                wait_bar(bar_q_full + 8, 0, abort, p.status);
-                tc_fence_after();
-                issue_s(1, 0);
+            // Order: S_0(0), S_1(0) (and, with two score buffers, S_0(1), S_1(1)),
+            // then per key tile j the batch of tile 0 (O_0 += P_0(j) V_j, then the
+            // next score product of tile 0: S_0(j+1), or S_0(j+2) with two score
+            // buffers) and then that of tile 1.  The tensor core runs one tile's
+            // batch while the other tile's softmax works, and the two softmax
+            // groups stay half a step apart.  With two score buffers the score
+            // product of a step is ready before the softmax reaches it, so the
+            // softmax does not wait for the tensor core between steps.
+            constexpr int kAhead = DB ? 2 : 1;       // score products issued ahead of the softmax
+            for (int j = 0; j < kAhead && j < n_kv; ++j) {
+                wait_kv(2 * j);
+                for (int ti = 0; ti < 2; ++ti) {
+                    if (j >= (ti ? n1 : n0)) continue;
+                    if (j == 0) {
+                        wait_bar(bar_q_full + 8 * ti, 0, abort, p.status);
+                        tc_fence_after();
+                    }
+                    issue_s(ti, j);
+                }
+                mma_commit_elect(bar_kv_empty + 8 * ((2 * j) % SLOTS));          // K_j
             }
-            mma_commit_elect(bar_kv_empty);                    // K_0 (slot 0)
             for (int j = 0; j < n_kv; ++j) {
                 for (int ti = 0; ti < 2; ++ti) {
                     const int n_i = ti ? n1 : n0;
                     if (j >= n_i) continue;
-                    wait_bar(bar_p_half + 8 * ti, j & 1, abort, p.status);
+                    // P_ti(j) sits in score buffer pb; its barriers' phase counts steps on that buffer
+                    const int pb = 2 * ti + (DB ? (j & 1) : 0);
+                    const uint32_t pph = (DB ? (j >> 1) : j) & 1;
+                    wait_bar(bar_p_half + 8 * pb, pph, abort, p.status);
                     tc_fence_after();
                     wait_kv(2 * j + 1);
                     issue_pv(ti, j, 0);
-                    wait_bar(bar_p_full + 8 * ti, j & 1, abort, p.status);
+                    wait_bar(bar_p_full + 8 * pb, pph, abort, p.status);
                     tc_fence_after();
                     issue_pv(ti, j, 1);
-                    if (j + 1 < n_i) {
-                        wait_kv(2 * j + 2);
-                        issue_s(ti, j + 1);
-                    } else {
-                        mma_commit_elect(bar_o_full + 8 * ti);
+                    if constexpr (DB) mma_commit_elect(bar_pv_done + 8 * ti);
+                    if (j + kAhead < n_i) {
+                        wait_kv(2 * (j + kAhead));
+                        issue_s(ti, j + kAhead);
                     }
+                    if (j + 1 == n_i) mma_commit_elect(bar_o_full + 8 * ti);
                 }
                 mma_commit_elect(bar_kv_empty + 8 * ((2 * j + 1) % SLOTS));            // V_j
-                if (j + 1 < n_kv) mma_commit_elect(bar_kv_empty + 8 * ((2 * j + 2) % SLOTS));   // K_{j+1}
+                if (j + kAhead < n_kv)
+                    mma_commit_elect(bar_kv_empty + 8 * ((2 * (j + kAhead)) % SLOTS));   // K_{j+kAhead}
             }
             // every product has completed before TMEM is released
             wait_bar(bar_o_full, 0, abort, p.status);

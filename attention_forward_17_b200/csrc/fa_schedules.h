@@ -27,7 +27,10 @@ struct Schedule {
                        // cluster launch control (tiles taken over from unlaunched CTAs)
     int alg;           // 0: one softmax pass over every key tile; 1: split-KV ping-pong
                        // (two softmax groups take alternate key tiles, merged at the end);
-                       // 2: two query tiles per CTA, P over S in TMEM, one issuer per tile
+                       // 2: two query tiles per CTA, P over S in TMEM, one score buffer per
+                       // tile; 3: the same with two score buffers per tile (scores of
+                       // the next key tile computed while the softmax works); 4, 5: as
+                       // 2, 3 with the sum of the bf16 weights on the tensor core
     int smem_bytes;    // dynamic shared memory per CTA
     int bn;            // rows of a key/value tile (128 except for algorithm 2)
     FwdLaunchFn launch[2];   // [causal]
@@ -79,19 +82,19 @@ constexpr Schedule make_pp_schedule() {
                     &setup_pp_both<D, EMU, SLOTS>};
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS, int BN>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT>
 cudaError_t launch_2q(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                       const CUtensorMap& to, const FwdParams& p, unsigned grid, cudaStream_t stream) {
-    fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN>
-        <<<grid, kThreads, Q2Cfg<D, SLOTS, BN>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+    fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN, DB, LT>
+        <<<grid, kThreads, Q2Cfg<D, SLOTS, BN, DB, LT>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS, int BN>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT>
 int setup_2q_one() {
-    auto* k = fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN>;
+    auto* k = fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN, DB, LT>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Q2Cfg<D, SLOTS, BN>::kSmemBytes) != cudaSuccess)
+                             Q2Cfg<D, SLOTS, BN, DB, LT>::kSmemBytes) != cudaSuccess)
         return -6;
     cudaFuncAttributes attr;
     if (cudaFuncGetAttributes(&attr, k) != cudaSuccess) return -6;
@@ -99,24 +102,26 @@ int setup_2q_one() {
     return 0;
 }
 
-template <int D, int EMU, int SLOTS, int BN>
+template <int D, int EMU, int SLOTS, int BN, bool DB, bool LT>
 int setup_2q_both() {
-    const int rc = setup_2q_one<D, false, EMU, SLOTS, BN>();
-    return rc ? rc : setup_2q_one<D, true, EMU, SLOTS, BN>();
+    const int rc = setup_2q_one<D, false, EMU, SLOTS, BN, DB, LT>();
+    return rc ? rc : setup_2q_one<D, true, EMU, SLOTS, BN, DB, LT>();
 }
 
-// Two query tiles per CTA (fa_fwd_2q_kernel), key tiles of BN rows.
-template <int D, int EMU, int SLOTS, int BN = 128>
+// Two query tiles per CTA (fa_fwd_2q_kernel), key tiles of BN rows: algorithm
+// 2 (one score buffer per tile), 3 (two, DB), 4 and 5 (as 2 and 3 with the sum
+// of the bf16 weights accumulated by the tensor core, LT).
+template <int D, int EMU, int SLOTS, int BN = 128, bool DB = false, bool LT = false>
 constexpr Schedule make_2q_schedule() {
     return Schedule{D,
                     EMU,
                     SLOTS,
                     0,
-                    2,
-                    Q2Cfg<D, SLOTS, BN>::kSmemBytes,
+                    2 + (DB ? 1 : 0) + (LT ? 2 : 0),
+                    Q2Cfg<D, SLOTS, BN, DB, LT>::kSmemBytes,
                     BN,
-                    {&launch_2q<D, false, EMU, SLOTS, BN>, &launch_2q<D, true, EMU, SLOTS, BN>},
-                    &setup_2q_both<D, EMU, SLOTS, BN>};
+                    {&launch_2q<D, false, EMU, SLOTS, BN, DB, LT>, &launch_2q<D, true, EMU, SLOTS, BN, DB, LT>},
+                    &setup_2q_both<D, EMU, SLOTS, BN, DB, LT>};
 }
 
 template <int D, bool CAUSAL, int EMU, int SLOTS, int PERSIST>

@@ -46,6 +46,7 @@ WORKLOADS = {
     # the same shape with unit-variance scores (the rescale-cost A/B against the line above)
     "b1_h32_n16384_d128": dict(B=1, H=32, N=16384, d=128, sigma_qk=1.0),
     "b2_h16_n4096_d128": dict(B=2, H=16, N=4096, d=128, sigma_qk=1.0),
+    "b1_h32_n16384_d64": dict(B=1, H=32, N=16384, d=64, sigma_qk=1.0),
     "b4_h8_n1024_d64": dict(B=4, H=8, N=1024, d=64, sigma_qk=1.0),
     # profiling size: Q, K, V, O = 4 x 64 MiB, above the L2, a short launch
     "b1_h64_n4096_d128": dict(B=1, H=64, N=4096, d=128, sigma_qk=1.0),
@@ -70,13 +71,14 @@ def load_peaks():
         return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
 
 
-KERNEL_FAMILY = {0: "fa_fwd_kernel", 1: "fa_fwd_pp_kernel", 2: "fa_fwd_2q_kernel"}
+KERNEL_FAMILY = {0: "fa_fwd_kernel", 1: "fa_fwd_pp_kernel", 2: "fa_fwd_2q_kernel", 3: "fa_fwd_2q_kernel",
+                 4: "fa_fwd_2q_kernel", 5: "fa_fwd_2q_kernel"}
 
 
 def measured_traffic(workload, algorithm=0):
     """DRAM bytes per non-causal launch from the committed ncu summary of the
     kernel family the headline runs (algorithm 0: fa_fwd_kernel, 1: the split-KV
-    ping-pong kernel, 2: the two-query-tile kernel), or None when that kernel's
+    ping-pong kernel, 2-5: the two-query-tile kernel), or None when that kernel's
     source changed since the counters were taken (or the summary does not cover
     this workload)."""
     if workload != DEFAULT_WORKLOAD:
@@ -645,15 +647,54 @@ def bench_sweep(args):
             torch.cuda.empty_cache()
 
 
+def bench_rescale(args):
+    """The cost of the lazy O rescale on the headline shape (B=1, H=32, N=16384,
+    d=128): for q, k ~ N(0, sigma^2) with sigma in {1, sqrt(3), 3}, both masks,
+    the table's schedule (or --schedule) is timed like the headline (--warmup,
+    then --steps launches, clocks sampled) and run once more with the rescale
+    counters on (fa_fwd_rescale_stats): one JSON line per (sigma, mask) with
+    TFLOP/s, TFLOP/s per GHz and the share of (warp, key tile) and (row, key
+    tile) steps that rescaled O."""
+    import numpy as np
+    import torch
+    import attention_forward_17_b200 as fa
+    import seeded_inputs as si
+    B, H, N, d = 1, 32, 16384, 128
+    for sigma in (1.0, 3.0 ** 0.5, 3.0):
+        bits = si.make_qkv(B, H, N, d, seed=0, sigma_qk=sigma)
+        q, k, v = (torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).cuda() for b in bits)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+        for c in (False, True):
+            kw = {} if args.schedule is None else {"schedule": args.schedule}
+            run = lambda: fa.fa_fwd(q, k, v, causal=c, out=o, lse=lse, **kw)
+            for _ in range(args.warmup):
+                run()
+            ms, clk = _event_loop(run, args.steps)
+            tf = flops(B, H, N, d, c) / (ms / 1e3) / 1e12
+            _, _, w, r, total = fa.rescale_stats(q, k, v, c, schedule=args.schedule)
+            print(json.dumps({"suite": "rescale", "B": B, "H": H, "N": N, "d": d, "qk_sigma": sigma,
+                              "mode": "causal" if c else "non-causal",
+                              "schedule": schedule_of(N, d, c, args.schedule), "tflops": tf,
+                              "tflops_per_ghz": tf / (clk["sm_mhz"] / 1e3) if clk.get("sm_mhz") else None,
+                              "clocks": clk, "warp_steps_rescaled": w, "row_steps_rescaled": r,
+                              "warp_steps": total, "warp_step_rate": w / total,
+                              "row_step_rate": r / (32 * total), "steps": args.steps,
+                              "warmup": args.warmup, "impl": "ours"}), flush=True)
+        del q, k, v, o, lse
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--suite", choices=["attention", "next", "sweep"], default="attention",
+    ap.add_argument("--suite", choices=["attention", "next", "sweep", "rescale"], default="attention",
                     help="'next' measures the kernels beyond the attention path, one line each; "
-                         "'sweep' the sequence-length sweep, one line per (d, N)")
+                         "'sweep' the sequence-length sweep, one line per (d, N); 'rescale' the "
+                         "lazy-rescale rate and its cost against the score range")
     ap.add_argument("--next", nargs="+", choices=["row_softmax", "gemm", "vector_add"],
                     default=["row_softmax", "gemm", "vector_add"],
                     help="kernels measured by --suite next")
@@ -678,6 +719,9 @@ def main():
     cfg = WORKLOADS[args.workload]
     if args.suite == "sweep":
         bench_sweep(args)
+        return
+    if args.suite == "rescale":
+        bench_rescale(args)
         return
     if args.suite == "next":
         for name in args.next:

@@ -126,8 +126,13 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
  *                     accumulators, merged per row at the end; 2 = two
  *                     128-row query tiles per CTA sharing every key/value
  *                     tile, P kept over the scores in tensor memory, one
- *                     tensor-core issuing thread per query tile, O stored
- *                     through shared memory with TMA), shared memory per CTA
+ *                     tensor-core issuing thread for both tiles in a fixed
+ *                     alternating order, O stored through shared memory with
+ *                     TMA; 3 = as 2 with two score buffers per query tile, so
+ *                     the scores of the next key tile are computed while the
+ *                     softmax works on the current one; 4, 5 = as 2, 3 with
+ *                     the sum of the bf16 weights accumulated by the tensor
+ *                     core, d = 64 only), shared memory per CTA
  *                     and rows of a key/value tile (128, or 64 / 192 for some
  *                     two-tile schedules) of schedule `id`; FA_ERR_ARG for an
  *                     unknown id.  Output pointers may be NULL.
@@ -160,8 +165,8 @@ int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float*
  *   dev_counts   device, two unsigned 64-bit counters, caller-owned, never
  *                cleared: [0] += (warp, key tile) steps at which at least one
  *                of the warp's 32 rows rescaled, [1] += (row, key tile)
- *                rescales.  Only the two-query-tile kernel (algorithm 2)
- *                counts; other schedules leave the counters unchanged.
+ *                rescales.  Only the two-query-tile kernel (algorithms 2
+ *                to 5) counts; other schedules leave the counters unchanged.
  *                NULL -> FA_ERR_NULL (after the checks of fa_fwd).
  * A diagnostic entry point: the atomics cost a little time.
  */

@@ -135,39 +135,41 @@ def test_model_flags_an_odd_ring_for_the_ping_pong_kernel():
 
 
 # ------------------------------------------------------------------ two-query-tile kernel
-def two_tile_issuer_events(n0, n1, release_k_early=False):
-    """The ring events of the two-query-tile kernel's single MMA issuer, in
-    program order, for key-tile counts n0 (tile 0) and n1 (tile 1): ("wait", L),
+def two_tile_issuer_events(n0, n1, ahead=1, release_k_early=False):
+    """The ring events of the two-query-tile kernel's MMA issuer, in program
+    order, for key-tile counts n0 (tile 0) and n1 (tile 1): ("wait", L),
     ("use", L), ("release", L) with L the load index (K_j = 2j, V_j = 2j+1).
-    release_k_early models a faulty variant that releases K_{j+1} right after
-    tile 0's score product."""
+    `ahead` is how many score products run ahead of the softmax (1 with one
+    score buffer per tile, 2 with two).  release_k_early models a faulty
+    variant that releases the next K tile right after tile 0's score product."""
     ev, waited = [], [-1]
 
-    def wait(ld):
-        if ld > waited[0]:
-            ev.append(("wait", ld))
-            waited[0] = ld
+    def wait(ld):                       # waits for every load up to ld, in order
+        while waited[0] < ld:
+            waited[0] += 1
+            ev.append(("wait", waited[0]))
 
     n_kv = max(n0, n1)
-    wait(0)
-    ev.append(("use", 0))
-    if n1 > 0:
-        ev.append(("use", 0))
-    ev.append(("release", 0))
+    for j in range(min(ahead, n_kv)):
+        wait(2 * j)
+        for n_i in (n0, n1):
+            if j < n_i:
+                ev.append(("use", 2 * j))
+        ev.append(("release", 2 * j))
     for j in range(n_kv):
         for ti, n_i in ((0, n0), (1, n1)):
             if j >= n_i:
                 continue
             wait(2 * j + 1)
             ev.append(("use", 2 * j + 1))
-            if j + 1 < n_i:
-                wait(2 * j + 2)
-                ev.append(("use", 2 * j + 2))
+            if j + ahead < n_i:
+                wait(2 * (j + ahead))
+                ev.append(("use", 2 * (j + ahead)))
                 if release_k_early and ti == 0:
-                    ev.append(("release", 2 * j + 2))
+                    ev.append(("release", 2 * (j + ahead)))
         ev.append(("release", 2 * j + 1))
-        if j + 1 < n_kv and not (release_k_early and j + 1 < n0):
-            ev.append(("release", 2 * j + 2))
+        if j + ahead < n_kv and not (release_k_early and j + ahead < n0):
+            ev.append(("release", 2 * (j + ahead)))
     return ev, 2 * n_kv
 
 
@@ -182,6 +184,10 @@ def two_tile_violations(n0, n1, slots, **kw):
             # a parity wait on load ld is sound once the slot's previous load was observed
             if ld >= slots and (ld - slots) not in landed:
                 bad += 1
+            # and the producer issues load ld only after load ld - slots was released:
+            # a release that comes later in the issuer's own order is a deadlock
+            if ld >= slots and (ld - slots) not in released:
+                bad += 1
             landed.add(ld)
         elif kind == "use":
             if ld not in landed or ld in released:
@@ -195,20 +201,63 @@ def two_tile_violations(n0, n1, slots, **kw):
     return bad
 
 
-def compiled_two_tile_depths():
-    return sorted({s["kv_slots"] for s in fa.schedules() if s["algorithm"] == 2})
+def compiled_two_tile_rings():
+    """(depth, score products ahead) of every compiled two-tile schedule."""
+    return sorted({(s["kv_slots"], 2 if s["algorithm"] in (3, 5) else 1)
+                   for s in fa.schedules() if s["algorithm"] >= 2})
 
 
-@pytest.mark.parametrize("slots", compiled_two_tile_depths())
-def test_two_tile_ring_is_sound(slots):
+@pytest.mark.parametrize("slots,ahead", compiled_two_tile_rings())
+def test_two_tile_ring_is_sound(slots, ahead):
     for n1 in range(0, 40):
-        # non-causal (equal counts), causal (tile 0 one key tile short), and a
-        # second tile past the end of the sequence (no keys)
-        for n0 in {n1, n1 - 1}:
+        # non-causal (equal counts), causal (tile 0 one to three key tiles short,
+        # for key tiles of 192, 128 and 64 rows), and a second tile past the end
+        # of the sequence (no keys)
+        for n0 in {n1, n1 - 1, n1 - 2}:
             if n0 >= 1:
-                assert two_tile_violations(n0, n1, slots) == 0, (n0, n1)
-        assert two_tile_violations(n1 + 1, 0, slots) == 0
+                assert two_tile_violations(n0, n1, slots, ahead=ahead) == 0, (n0, n1)
+        assert two_tile_violations(n1 + 1, 0, slots, ahead=ahead) == 0
+
+
+def test_model_flags_a_shallow_ring_with_two_score_buffers():
+    # K_{j+2} is needed while V_j is still unreleased: three slots deadlock
+    assert sum(two_tile_violations(n, n, 3, ahead=2) for n in range(3, 20)) > 0
+    assert all(s["kv_slots"] >= 4 for s in fa.schedules() if s["algorithm"] in (3, 5))
 
 
 def test_model_flags_an_early_key_release():
-    assert sum(two_tile_violations(n, n, 5, release_k_early=True) for n in range(2, 20)) > 0
+    for ahead in (1, 2):
+        assert sum(two_tile_violations(n, n, 5, ahead=ahead, release_k_early=True)
+                   for n in range(3, 20)) > 0
+
+
+# ------------------------------------------------------------------ P barriers of the two-tile kernel
+def p_barrier_unsound_waits(n, ahead, nbufs):
+    """Parity waits of the issuer on the P barriers that the softmax can have
+    run two phases past.  The softmax is modelled as fast as its inputs allow:
+    it releases P(k) as soon as S(k) exists, and S(k) is issued in the prologue
+    (k < ahead) or right after the issuer consumed P(k - ahead).  P(k) lives on
+    barrier k % nbufs (phase k // nbufs).  When the issuer waits for P(j) it has
+    consumed P(0..j-1), so the softmax can have released P(0 .. j-1+ahead); the
+    wait is unsound if that includes the next phase of the same barrier, P(j+nbufs)."""
+    bad = 0
+    for j in range(n):
+        released_up_to = min(n - 1, j - 1 + ahead)
+        if j + nbufs <= released_up_to:
+            bad += 1
+    return bad
+
+
+def test_p_barriers_cannot_run_two_phases_ahead():
+    for s in fa.schedules():
+        if s["algorithm"] < 2:
+            continue
+        ahead = nbufs = 2 if s["algorithm"] in (3, 5) else 1
+        for n in range(1, 40):
+            assert p_barrier_unsound_waits(n, ahead, nbufs) == 0, (s, n)
+
+
+def test_model_flags_one_p_barrier_with_two_score_buffers():
+    # the first version of the double-buffered kernel kept one P barrier per tile:
+    # its issuer's waits ran out of time once the softmax got a step ahead
+    assert sum(p_barrier_unsound_waits(n, 2, 1) for n in range(3, 20)) > 0

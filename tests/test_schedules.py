@@ -73,7 +73,7 @@ def test_two_tile_kernel_edges(cuda_device):
     # the two-query-tile kernel on shapes that exercise its pairing: one row, a
     # lone first tile, a pair whose second tile is ragged or empty (odd tile
     # counts), several slices, both masks
-    sched = [s for s in _schedules() if s["algorithm"] == 2]
+    sched = [s for s in _schedules() if s["algorithm"] >= 2]
     assert sched, "no two-query-tile schedule compiled"
     for s in sched:
         d = s["d"]
