@@ -21,7 +21,7 @@ const Schedule kD128[] = {
     make_schedule<128, 4, 5, 2>(), make_schedule<128, 4, 4, 2>(),
     make_pp_schedule<128, 4, 4>(), make_pp_schedule<128, 0, 4>(),
     make_2q_schedule<128, 4, 5>(), make_2q_schedule<128, 8, 5>(), make_2q_schedule<128, 2, 5>(),
-    make_2q_schedule<128, 0, 5>(), make_2q_schedule<128, 4, 3>(),
+    make_2q_schedule<128, 0, 5>(), make_2q_schedule<128, 4, 3>(), make_2q_schedule<128, 3, 5>(),
     make_2q_schedule<128, 4, 8, 64>(),
     make_2q_schedule<128, 4, 8, 64, true>(), make_2q_schedule<128, 0, 8, 64, true>(),
 };

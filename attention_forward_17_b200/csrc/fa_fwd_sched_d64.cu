@@ -21,8 +21,8 @@ const Schedule kD64[] = {
     make_2q_schedule<64, 4, 4>(),
     make_2q_schedule<64, 4, 8, 64>(), make_2q_schedule<64, 4, 8, 192>(),
     make_2q_schedule<64, 4, 8, 64, true>(),
-    make_2q_schedule<64, 4, 8, 128, false, true>(), make_2q_schedule<64, 2, 8, 128, false, true>(),
-    make_2q_schedule<64, 4, 8, 64, true, true>(),
+    make_2q_schedule<64, 4, 8, 128, false, true>(),
+    make_2q_schedule<64, 4, 8, 64, true, true>(), make_2q_schedule<64, 3, 8, 128, false, true>(),
 };
 }  // namespace
 

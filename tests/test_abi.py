@@ -155,7 +155,7 @@ def test_schedule_registry():
         bufs = 2 if alg in (3, 5) else 1      # score buffers per query tile
         do = d + 16 if alg in (4, 5) else d   # O columns (16 more when the tensor core sums l^)
         assert 2 * bufs * bn + 2 * do <= 512 and (bn == 128 or (alg >= 2 and bn in (64, 192)))
-        assert d in (64, 128) and emu in (0, 2, 4, 8) and persist in (0, 1, 2)
+        assert d in (64, 128) and emu in (0, 2, 3, 4, 8) and persist in (0, 1, 2)
         assert alg in (0, 1, 2, 3, 4, 5) and 0 < smem <= 232448
         # the one-tile kernels need four slots for sound parity waits; the
         # two-tile kernel's issuers observe every load in order, so any depth >= 2
