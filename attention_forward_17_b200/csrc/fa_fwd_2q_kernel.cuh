@@ -281,8 +281,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t c2 = f2(cl, cl);
 
 
-        float m = -INFINITY;                      // running max of c*s (stale by < 8)
+        float m = -INFINITY;                      // running max of c*s (stale by up to kRescaleTau)
         float l = 0.f, lh = 0.f;                  // sums of the weights: fp32, and bf16-rounded
+        constexpr int kHW = C::kHalfWords;        // P words released at a time (BN/2 keys)
         for (int j = 0; j < n_i; ++j) {
             // score buffer of this step: with DB, S_i(j) sits in buffer j % 2
             const int sb = DB ? (j & 1) : 0;
@@ -292,59 +293,93 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool masked =
                 (j * BN + BN > p.N) || (CAUSAL && j * BN + BN - 1 > q0);
             const int lim = (CAUSAL ? min(p.N, row + 1) : p.N) - j * BN;   // keys >= lim are masked
-            // Scores of this row, 32 columns at a time (kRegCols held in
-            // registers; wider key tiles are read twice: once for the maximum,
-            // once for the exponentials).
+            // Scores of this row (kRegCols held in registers; wider key tiles are
+            // read twice: once for the maximum, once for the exponentials).
             constexpr int kRegCols = BN <= 128 ? BN : BN / 2;
             uint32_t s[kRegCols];
-            const auto load_cols = [&](int c0) {
+            // loads columns c0 .. c0+n-1 into s[i0 ..]; the caller waits for them
+            const auto issue_loads = [&](int c0, int i0, int n) {
 #pragma unroll
-                for (int q = 0; q < kRegCols / 32; ++q)
-                    tmem_ld32(t_s + c0 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * q]));
-                tmem_wait_ld();
-                // the wait carries no register operands: pin the loaded values after it
+                for (int q = 0; q < n / 32; ++q)
+                    tmem_ld32(t_s + c0 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&s[i0 + 32 * q]));
+            };
+            // after tcgen05.wait::ld: pin s[i0 .. i0+n) after the wait (it carries no
+            // register operands) and mask the keys past the row's limit
+            const auto settle = [&](int c0, int i0, int n) {
 #pragma unroll
-                for (int q = 0; q < kRegCols / 32; ++q)
-                    reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[32 * q]));
+                for (int q = 0; q < n / 32; ++q)
+                    reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[i0 + 32 * q]));
                 if (masked) {
 #pragma unroll
-                    for (int k = 0; k < kRegCols; ++k)
-                        if (c0 + k >= lim) s[k] = __float_as_uint(-INFINITY);
+                    for (int k = 0; k < n; ++k)
+                        if (c0 + k >= lim) s[i0 + k] = __float_as_uint(-INFINITY);
                 }
             };
-            // row maximum: independent chains of three-way maxima over 16 keys each,
-            // then a short tree
+            // row maximum: independent chains of three-way maxima over 16 keys each
+            // (group g of 16 keys on chain g % 8), then a short tree
             float x[8];
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) x[ch] = -INFINITY;
+            const auto max_groups = [&](int g0, int i0, int ng) {
 #pragma unroll
-            for (int c0 = 0; c0 < BN; c0 += kRegCols) {
-                if (BN > 128 || c0 == 0) load_cols(c0);
-#pragma unroll
-                for (int ch = 0; ch < kRegCols / 16; ++ch) {
-                    float& xc = x[(c0 / 16 + ch) & 7];
+                for (int g = 0; g < ng; ++g) {
+                    float& xc = x[(g0 + g) & 7];
 #pragma unroll
                     for (int k = 0; k < 16; k += 2)
-                        xc = max3f(xc, __uint_as_float(s[16 * ch + k]), __uint_as_float(s[16 * ch + k + 1]));
+                        xc = max3f(xc, __uint_as_float(s[i0 + 16 * g + k]), __uint_as_float(s[i0 + 16 * g + k + 1]));
                 }
-            }
-            const float mn =
-                fmaxf(max3f(x[0], x[1], x[2]), max3f(x[3], x[4], fmaxf(x[5], max3f(x[6], x[7], x[7])))) * cl;
-            const bool grow = mn > m + kRescaleTau;
-            float alpha = 1.f;
-            if (grow) {
-                alpha = ex2_approx(m - mn);
-                m = mn;
-                l *= alpha;
-                lh *= alpha;
-            }
-            // Lazy rescale of this row of O_i.  O_i holds the products of steps
-            // < j: with one score buffer they have all completed (S_i(j) was
-            // issued after PV_i(j-1)); with two, S_i(j) was issued before
-            // PV_i(j-1), so the rescale first waits for that product.  The stores
-            // complete before the first release of P below (tcgen05.wait::st).
-            const bool need = grow && j > 0;
-            if (__any_sync(0xffffffffu, need)) {
+            };
+            const auto row_max = [&]() {
+                return fmaxf(max3f(x[0], x[1], x[2]), max3f(x[3], x[4], fmaxf(x[5], max3f(x[6], x[7], x[7])))) * cl;
+            };
+            // Weights 2^(c*s - m), their sums, and P as bf16 pairs (word k = keys
+            // 2k, 2k+1) for half h of the keys (BN/2 keys, their scores at s[i0 ..]).
+            uint64_t la0 = 0, la1 = 0;
+            float hl0 = 0.f, hh0 = 0.f, hl1 = 0.f, hh1 = 0.f;
+            const auto weights_half = [&](int h, int i0, uint64_t negm, uint32_t (&pw)[kHW]) {
+#pragma unroll
+                for (int k = 0; k < kHW; ++k) {
+                    const int kk = kHW * h + k;                          // word index in the row
+                    const int sk = i0 + 2 * k;                           // its keys in s[]
+                    const uint64_t x2v = fma2(f2(__uint_as_float(s[sk]), __uint_as_float(s[sk + 1])), c2, negm);
+                    float e0, e1, p0, p1;
+                    f2_split(x2v, e0, e1);
+                    if (EMU > 0 && (kk % (EMU > 0 ? EMU : 1)) == EMU - 1) {
+                        exp2_poly2(e0, e1, p0, p1);
+                    } else {
+                        p0 = ex2_approx(e0);
+                        p1 = ex2_approx(e1);
+                    }
+                    const uint32_t w = pack_bf16x2(p0, p1);
+                    const uint64_t pr = f2(p0, p1);
+                    // the bf16 halves of w added to fp32 sums directly (mixed-precision
+                    // adds), unless the tensor core sums them (LT)
+                    if (k & 1) {
+                        la1 = add2(la1, pr);
+                        if constexpr (!LT) add_bf16x2_halves(hl1, hh1, w);
+                    } else {
+                        la0 = add2(la0, pr);
+                        if constexpr (!LT) add_bf16x2_halves(hl0, hh0, w);
+                    }
+                    pw[k] = w;
+                }
+            };
+            // Stores half h of P over the first BN/2 columns of S_i, whose scores this
+            // thread has already read, and releases it to the issuer: the product
+            // with the first half runs while the second half is computed.
+            const auto release_half = [&](int h, uint32_t (&pw)[kHW]) {
+                store_words<kHW>(t_p + kHW * h, pw);
+                tc_fence_before();
+                mbar_arrive((h == 0 ? bar_p_half : bar_p_full) + 8 * (2 * ti + sb));
+            };
+            // Lazy rescale of this row of O_i (warp-collective TMEM round trip when
+            // any row of the warp needs it).  O_i holds the products of steps < j:
+            // with one score buffer they have all completed (S_i(j) was issued after
+            // PV_i(j-1)); with two, S_i(j) was issued before PV_i(j-1), so the
+            // rescale first waits for that product.  The stores complete before the
+            // first release of P (tcgen05.wait::st).
+            const auto rescale_o = [&](bool need, float alpha) {
+                if (!__any_sync(0xffffffffu, need)) return;
                 if constexpr (DB) {
                     wait_bar(bar_pv_done + 8 * ti, (j - 1) & 1, abort, p.status);
                     tc_fence_after();
@@ -377,50 +412,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                     reg_fence16(o);
                     tmem_st16(t_o + D, o);
                 }
+            };
+            uint32_t pw[kHW];
+#pragma unroll
+            for (int c0 = 0; c0 < BN; c0 += kRegCols) {
+                if (BN > 128 || c0 == 0) {
+                    issue_loads(c0, 0, kRegCols);
+                    tmem_wait_ld();
+                    settle(c0, 0, kRegCols);
+                }
+                max_groups(c0 / 16, 0, kRegCols / 16);
             }
+            const float mn = row_max();
+            const bool grow = mn > m + kRescaleTau;
+            float alpha = 1.f;
+            if (grow) {
+                alpha = ex2_approx(m - mn);
+                m = mn;
+                l *= alpha;
+                lh *= alpha;
+            }
+            rescale_o(grow && j > 0, alpha);
             const float u = (m == -INFINITY) ? 0.f : m;
             const uint64_t negm = f2(-u, -u);
-            // Weights 2^(c*s - m), their sums, and P as bf16 pairs (word k = keys
-            // 2k, 2k+1), in two halves of BN/2 keys: each half is stored to TMEM
-            // and released on its own barrier, so the product with the first
-            // half runs while the second half is computed.  P goes over the
-            // first BN/2 columns of S_i, whose scores this thread has already read.
-            constexpr int kHW = C::kHalfWords;
-            uint64_t la0 = 0, la1 = 0;
-            float hl0 = 0.f, hh0 = 0.f, hl1 = 0.f, hh1 = 0.f;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                if constexpr (BN > 128) load_cols(h * kRegCols);
-                uint32_t pw[kHW];
-#pragma unroll
-                for (int k = 0; k < kHW; ++k) {
-                    const int kk = kHW * h + k;                          // word index in the row
-                    const int sk = BN > 128 ? 2 * k : 2 * kk;            // its keys in s[]
-                    const uint64_t x2v = fma2(f2(__uint_as_float(s[sk]), __uint_as_float(s[sk + 1])), c2, negm);
-                    float e0, e1, p0, p1;
-                    f2_split(x2v, e0, e1);
-                    if (EMU > 0 && (kk % (EMU > 0 ? EMU : 1)) == EMU - 1) {
-                        exp2_poly2(e0, e1, p0, p1);
-                    } else {
-                        p0 = ex2_approx(e0);
-                        p1 = ex2_approx(e1);
-                    }
-                    const uint32_t w = pack_bf16x2(p0, p1);
-                    const uint64_t pr = f2(p0, p1);
-                    // the bf16 halves of w added to fp32 sums directly (mixed-precision
-                    // adds), unless the tensor core sums them (LT)
-                    if (k & 1) {
-                        la1 = add2(la1, pr);
-                        if constexpr (!LT) add_bf16x2_halves(hl1, hh1, w);
-                    } else {
-                        la0 = add2(la0, pr);
-                        if constexpr (!LT) add_bf16x2_halves(hl0, hh0, w);
-                    }
-                    pw[k] = w;
+                if constexpr (BN > 128) {
+                    issue_loads(h * kRegCols, 0, kRegCols);
+                    tmem_wait_ld();
+                    settle(h * kRegCols, 0, kRegCols);
                 }
-                store_words<kHW>(t_p + kHW * h, pw);
-                tc_fence_before();
-                mbar_arrive((h == 0 ? bar_p_half : bar_p_full) + 8 * (2 * ti + sb));
+                weights_half(h, BN > 128 ? 0 : h * (BN / 2), negm, pw);
+                release_half(h, pw);
             }
             float v0, v1;
             f2_split(add2(la0, la1), v0, v1);
