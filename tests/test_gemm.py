@@ -2,7 +2,9 @@
 oracle on the same seeded bf16 inputs: single tiles, ragged M / N / K tails,
 more tiles than SMs (each CTA cycles through both tensor-memory accumulators
 and the shared-memory ring several times), K = 0, all three epilogues, and
-sampled entries of the 8192^3 problem the benchmark times.
+sampled entries of the 8192^3 problem the benchmark times.  Problems of at
+most 128 rows (and K = 0) run the one-SM kernel; the others run 256-row tiles
+over SM pairs, including pairs whose second CTA holds one valid row or none.
 
 Bound per element: C is rounded to bf16 (relative error <= 2^-9); fp32
 accumulation of at most K exact bf16 products and erff add well under 1e-3
@@ -45,7 +47,8 @@ SHAPES = [
     (1, 8, 8),           # smallest legal problem
     (300, 520, 200),     # ragged M, N (last column block is 8 wide), K (last block 8 deep)
     (257, 264, 72),
-    (640, 768, 1024),    # 16 K blocks: the 4-stage ring wraps four times
+    (129, 136, 24),      # one 256-row pair tile: the second CTA holds a single valid row
+    (640, 768, 1024),    # 16 K blocks: the stage rings wrap several times
 ]
 
 
