@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 //                (the odd CTA's remotely) once they have read accumulator b.
 // Before exit each CTA waits for the last arrivals addressed to it, then the
 // pair meets at a cluster barrier and frees its TMEM.
-constexpr int k2BM = 256, k2Stages = 6;
+constexpr int k2BM = 256, k2Stages = 7;
 constexpr int k2ABytes = 128 * kBK * 2;           // 16 KiB: this CTA's 128 rows of A
 constexpr int k2BBoxes = 2;                       // this CTA's 128 columns of B: 2 boxes of 64
 constexpr int k2StageBytes = k2ABytes + k2BBoxes * kBBoxBytes;   // 32 KiB
@@ -406,7 +406,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (even CTA)
-        if (rank == 0 && lane == 0) {
+        // The whole warp runs the loop (converged, waits included); one elected
+        // lane issues each product and commit.
+        if (rank == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(k2BM, kBN, true);
             int s = 0, tl = 0;
             uint32_t ph = 0;
@@ -423,16 +425,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t b_st = a_st + k2ABytes;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
-                        mma_ss_pair(d, smem_desc_sw128(a_st + 32 * kk, 16, 1024),
+                        mma_ss_pair_elect(d, smem_desc_sw128(a_st + 32 * kk, 16, 1024),
                                     smem_desc_sw128(b_st + 2048 * kk, kBBoxBytes, 1024), idesc,
                                     (kb | kk) != 0 ? 1u : 0u);
-                    mma_commit_pair(empty(s), 0x3);
+                    mma_commit_pair_elect(empty(s), 0x3);
                     if (++s == k2Stages) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
-                mma_commit_pair(acc_full(buf), 0x3);
+                mma_commit_pair_elect(acc_full(buf), 0x3);
             }
             // both CTAs' epilogues have released every accumulator (their remote
             // arrivals have landed) before this CTA may exit: wait as if for the

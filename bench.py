@@ -554,7 +554,7 @@ def bench_gemm(args):
                        "l2": "A, B, C = 384 MiB, above L2"},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16"],
                          "unit": "TFLOP/s", "frac": tf / peaks["bf16"],
-                         "traffic": profile_traffic("gemm_kernel_m8192_n8192_k8192_ncu.md",
+                         "traffic": profile_traffic("gemm2_kernel_m8192_n8192_k8192_ncu.md",
                                                     "attention_forward_17_b200/csrc/gemm_bias_gelu.cu"),
                          "algorithmic_flops_per_launch": flop,
                          "peak_source": peaks["source"] + " bf16 burst (cuBLAS 8192^3)"},
