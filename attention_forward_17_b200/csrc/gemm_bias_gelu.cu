@@ -22,7 +22,7 @@
 //               fp32, rounds to bf16 (nearest-even) and stores 16-byte
 //               vectors.  With two accumulators the epilogue of tile t runs
 //               while the tensor core works on tile t + 1.
-// Tiles are visited in groups of 16 row blocks so the CTAs in flight share
+// Tiles are visited in groups of 8 row blocks so the CTAs in flight share
 // A and B panels in L2.
 //
 // That one-SM kernel runs problems of at most 128 rows (and K = 0).  Larger
@@ -51,7 +51,7 @@ constexpr int kBBoxBytes = 64 * kBK * 2;          // 8 KiB: 64 N columns x 64 K 
 constexpr int kStageBytes = kABytes + 4 * kBBoxBytes;
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
-constexpr int kGroupM = 16;
+constexpr int kGroupM = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBarOff = kStages * kStageBytes;
 constexpr int kSmemBytes = 1024 + kBarOff + 256;  // 1 KiB for aligning the ring
