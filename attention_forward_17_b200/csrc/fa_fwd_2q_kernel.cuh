@@ -106,7 +106,6 @@ struct Q2Cfg {
     }
     static constexpr uint32_t kColO = 2 * kSBufs * BN;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr int kHalfWords = BN / 4;               // P words released at a time
     static_assert(kSmemBytes <= 232448, "shared memory per CTA (227 KiB)");
     static_assert(kColO + 2 * kDO <= kTmemCols, "score and output buffers in TMEM");
     static_assert(kKVBoxBytes % 1024 == 0, "slots on 1024-byte boundaries (128-byte swizzle)");
@@ -184,12 +183,22 @@ __device__ __forceinline__ void map_pair(const FwdParams& p, int n_pair, int id,
     }
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                      const FwdParams p) {
     using C = Q2Cfg<D, SLOTS, BN, DB, LT>;
+    // P is released in two parts of kW0 and kW1 words (two keys a word): halves,
+    // or with P34 the first three quarters of the keys and then the last quarter.
+    // The product with the first part then runs while the last quarter's weights
+    // are computed and ends about when they are released, so only a quarter of
+    // the key tile's P.V product follows the softmax's last release (instead of
+    // half): the chain softmax -> P.V -> next scores -> softmax that bounds a
+    // tile's step gets shorter by a quarter of a P.V product.
+    static_assert(!P34 || BN == 128, "three-quarter release: key tiles of 128 rows");
+    constexpr int kW0 = P34 ? 3 * BN / 8 : BN / 4;
+    constexpr int kW1 = BN / 2 - kW0;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -283,7 +292,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         float m = -INFINITY;                      // running max of c*s (stale by up to kRescaleTau)
         float l = 0.f, lh = 0.f;                  // sums of the weights: fp32, and bf16-rounded
-        constexpr int kHW = C::kHalfWords;        // P words released at a time (BN/2 keys)
         for (int j = 0; j < n_i; ++j) {
             // score buffer of this step: with DB, S_i(j) sits in buffer j % 2
             const int sb = DB ? (j & 1) : 0;
@@ -333,13 +341,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return fmaxf(max3f(x[0], x[1], x[2]), max3f(x[3], x[4], fmaxf(x[5], max3f(x[6], x[7], x[7])))) * cl;
             };
             // Weights 2^(c*s - m), their sums, and P as bf16 pairs (word k = keys
-            // 2k, 2k+1) for half h of the keys (BN/2 keys, their scores at s[i0 ..]).
+            // 2k, 2k+1) for part h of the keys (2 kW0 or 2 kW1 keys, their scores
+            // at s[i0 ..]).
             uint64_t la0 = 0, la1 = 0;
             float hl0 = 0.f, hh0 = 0.f, hl1 = 0.f, hh1 = 0.f;
-            const auto weights_half = [&](int h, int i0, uint64_t negm, uint32_t (&pw)[kHW]) {
+            const auto weights_half = [&](int h, int i0, uint64_t negm, uint32_t (&pw)[kW0]) {
 #pragma unroll
-                for (int k = 0; k < kHW; ++k) {
-                    const int kk = kHW * h + k;                          // word index in the row
+                for (int k = 0; k < (h ? kW1 : kW0); ++k) {
+                    const int kk = (h ? kW0 : 0) + k;                    // word index in the row
                     const int sk = i0 + 2 * k;                           // its keys in s[]
                     const uint64_t x2v = fma2(f2(__uint_as_float(s[sk]), __uint_as_float(s[sk + 1])), c2, negm);
                     float e0, e1, p0, p1;
@@ -364,11 +373,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pw[k] = w;
                 }
             };
-            // Stores half h of P over the first BN/2 columns of S_i, whose scores this
-            // thread has already read, and releases it to the issuer: the product
-            // with the first half runs while the second half is computed.
-            const auto release_half = [&](int h, uint32_t (&pw)[kHW]) {
-                store_words<kHW>(t_p + kHW * h, pw);
+            // Stores part h of P over the first BN/2 columns of S_i, whose scores
+            // this thread has already read, and releases it to the issuer: the
+            // product with the first part runs while the second is computed.
+            const auto release_half = [&](int h, uint32_t (&pw)[kW0]) {
+                if (h == 0)
+                    store_words<kW0>(t_p, pw);
+                else
+                    store_words<kW1>(t_p + kW0, *reinterpret_cast<uint32_t(*)[kW1]>(&pw[0]));
                 tc_fence_before();
                 mbar_arrive((h == 0 ? bar_p_half : bar_p_full) + 8 * (2 * ti + sb));
             };
@@ -413,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st16(t_o + D, o);
                 }
             };
-            uint32_t pw[kHW];
+            uint32_t pw[kW0];
 #pragma unroll
             for (int c0 = 0; c0 < BN; c0 += kRegCols) {
                 if (BN > 128 || c0 == 0) {
@@ -442,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_wait_ld();
                     settle(h * kRegCols, 0, kRegCols);
                 }
-                weights_half(h, BN > 128 ? 0 : h * (BN / 2), negm, pw);
+                weights_half(h, BN > 128 ? 0 : 2 * (h ? kW0 : 0), negm, pw);
                 release_half(h, pw);
             }
             float v0, v1;
@@ -583,8 +595,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 mma_commit_elect(bar_s_full + 8 * (2 * ti + sb));
             };
-            // O_ti += P_ti(j) V_j for the keys of half h (BN/2 keys), P from TMEM
-            // (8 columns per 16 keys)
+            // O_ti += P_ti(j) V_j for the keys of part h (2 kW0 or 2 kW1 keys), P
+            // from TMEM (8 columns per 16 keys)
             const auto issue_pv = [&](int ti, int j, int h) {
                 const uint32_t v_addr = slot_addr(2 * j + 1);
                 // LT: V's second 64-column chunk (one chunk stride, LBO, further on)
@@ -594,8 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t a_p = tmem + C::col_s(ti, DB ? (j & 1) : 0);
                 const uint32_t d_o = tmem + C::kColO + static_cast<uint32_t>(C::kDO) * ti;
 #pragma unroll
-                for (int k4 = 0; k4 < BN / 32; ++k4) {
-                    const int kk = (BN / 32) * h + k4;
+                for (int k4 = 0; k4 < (h ? kW1 : kW0) / 8; ++k4) {
+                    const int kk = (h ? kW0 / 8 : 0) + k4;          // 16 keys (8 P words) each
                     mma_ts_elect(d_o, a_p + kk * 8, b_v + kk * (2048 >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 }
             };

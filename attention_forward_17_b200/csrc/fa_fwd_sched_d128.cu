@@ -24,6 +24,8 @@ const Schedule kD128[] = {
     make_2q_schedule<128, 0, 5>(), make_2q_schedule<128, 4, 3>(), make_2q_schedule<128, 3, 5>(),
     make_2q_schedule<128, 4, 8, 64>(),
     make_2q_schedule<128, 4, 8, 64, true>(), make_2q_schedule<128, 0, 8, 64, true>(),
+    make_2q_schedule<128, 4, 5, 128, false, false, true>(), make_2q_schedule<128, 3, 5, 128, false, false, true>(),
+    make_2q_schedule<128, 0, 5, 128, false, false, true>(),
 };
 }  // namespace
 

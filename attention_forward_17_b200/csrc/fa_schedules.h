@@ -30,9 +30,10 @@ struct Schedule {
                        // 2: two query tiles per CTA, P over S in TMEM, one score buffer per
                        // tile; 3: the same with two score buffers per tile (scores of
                        // the next key tile computed while the softmax works); 4, 5: as
-                       // 2, 3 with the sum of the bf16 weights on the tensor core
+                       // 2, 3 with the sum of the bf16 weights on the tensor core; 6 to 9:
+                       // as 2 to 5 with P released as 3/4 and then 1/4 of the keys
     int smem_bytes;    // dynamic shared memory per CTA
-    int bn;            // rows of a key/value tile (128 except for algorithm 2)
+    int bn;            // rows of a key/value tile (128 except for the two-query-tile algorithms)
     FwdLaunchFn launch[2];   // [causal]
     int (*setup)();          // shared-memory opt-in and register check, both modes
 };
@@ -82,17 +83,17 @@ constexpr Schedule make_pp_schedule() {
                     &setup_pp_both<D, EMU, SLOTS>};
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34>
 cudaError_t launch_2q(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                       const CUtensorMap& to, const FwdParams& p, unsigned grid, cudaStream_t stream) {
-    fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN, DB, LT>
+    fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN, DB, LT, P34>
         <<<grid, kThreads, Q2Cfg<D, SLOTS, BN, DB, LT>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34>
 int setup_2q_one() {
-    auto* k = fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN, DB, LT>;
+    auto* k = fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN, DB, LT, P34>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Q2Cfg<D, SLOTS, BN, DB, LT>::kSmemBytes) != cudaSuccess)
         return -6;
@@ -102,26 +103,27 @@ int setup_2q_one() {
     return 0;
 }
 
-template <int D, int EMU, int SLOTS, int BN, bool DB, bool LT>
+template <int D, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34>
 int setup_2q_both() {
-    const int rc = setup_2q_one<D, false, EMU, SLOTS, BN, DB, LT>();
-    return rc ? rc : setup_2q_one<D, true, EMU, SLOTS, BN, DB, LT>();
+    const int rc = setup_2q_one<D, false, EMU, SLOTS, BN, DB, LT, P34>();
+    return rc ? rc : setup_2q_one<D, true, EMU, SLOTS, BN, DB, LT, P34>();
 }
 
 // Two query tiles per CTA (fa_fwd_2q_kernel), key tiles of BN rows: algorithm
-// 2 (one score buffer per tile), 3 (two, DB), 4 and 5 (as 2 and 3 with the sum
-// of the bf16 weights accumulated by the tensor core, LT).
-template <int D, int EMU, int SLOTS, int BN = 128, bool DB = false, bool LT = false>
+// 2 (one score buffer per tile), + 1 with two score buffers per tile (DB), + 2
+// with the sum of the bf16 weights accumulated by the tensor core (LT), + 4 with
+// P released as three quarters and one quarter of the keys (P34): 2 to 9.
+template <int D, int EMU, int SLOTS, int BN = 128, bool DB = false, bool LT = false, bool P34 = false>
 constexpr Schedule make_2q_schedule() {
     return Schedule{D,
                     EMU,
                     SLOTS,
                     0,
-                    2 + (DB ? 1 : 0) + (LT ? 2 : 0),
+                    2 + (DB ? 1 : 0) + (LT ? 2 : 0) + (P34 ? 4 : 0),
                     Q2Cfg<D, SLOTS, BN, DB, LT>::kSmemBytes,
                     BN,
-                    {&launch_2q<D, false, EMU, SLOTS, BN, DB, LT>, &launch_2q<D, true, EMU, SLOTS, BN, DB, LT>},
-                    &setup_2q_both<D, EMU, SLOTS, BN, DB, LT>};
+                    {&launch_2q<D, false, EMU, SLOTS, BN, DB, LT, P34>, &launch_2q<D, true, EMU, SLOTS, BN, DB, LT, P34>},
+                    &setup_2q_both<D, EMU, SLOTS, BN, DB, LT, P34>};
 }
 
 template <int D, bool CAUSAL, int EMU, int SLOTS, int PERSIST>

@@ -71,7 +71,7 @@ def load_peaks():
         return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
 
 
-KERNEL_FAMILY = {0: "fa_fwd_kernel", 1: "fa_fwd_pp_kernel", **{a: "fa_fwd_2q_kernel" for a in range(2, 6)}}
+KERNEL_FAMILY = {0: "fa_fwd_kernel", 1: "fa_fwd_pp_kernel", **{a: "fa_fwd_2q_kernel" for a in range(2, 10)}}
 
 
 def measured_traffic(workload, algorithm=0):

@@ -205,7 +205,7 @@ def two_tile_violations(n0, n1, slots, **kw):
 
 def compiled_two_tile_rings():
     """(depth, score products ahead) of every compiled two-tile schedule."""
-    return sorted({(s["kv_slots"], 2 if s["algorithm"] in (3, 5) else 1)
+    return sorted({(s["kv_slots"], 2 if (s["algorithm"] - 2) & 1 else 1)
                    for s in fa.schedules() if s["algorithm"] >= 2})
 
 
@@ -224,7 +224,7 @@ def test_two_tile_ring_is_sound(slots, ahead):
 def test_model_flags_a_shallow_ring_with_two_score_buffers():
     # K_{j+2} is needed while V_j is still unreleased: three slots deadlock
     assert sum(two_tile_violations(n, n, 3, ahead=2) for n in range(3, 20)) > 0
-    assert all(s["kv_slots"] >= 4 for s in fa.schedules() if s["algorithm"] in (3, 5))
+    assert all(s["kv_slots"] >= 4 for s in fa.schedules() if s["algorithm"] >= 2 and (s["algorithm"] - 2) & 1)
 
 
 def test_model_flags_an_early_key_release():
@@ -254,7 +254,7 @@ def test_p_barriers_cannot_run_two_phases_ahead():
     for s in fa.schedules():
         if s["algorithm"] < 2:
             continue
-        ahead = nbufs = 2 if s["algorithm"] in (3, 5) else 1
+        ahead = nbufs = 2 if (s["algorithm"] - 2) & 1 else 1
         for n in range(1, 40):
             assert p_barrier_unsound_waits(n, ahead, nbufs) == 0, (s, n)
 
