@@ -22,12 +22,12 @@ struct ScheduleTableEntry {
 };
 
 constexpr ScheduleTableEntry kScheduleTable[] = {
-    {128, 0, 2048, 3, 5, 1, 0, 2, 128},
-    {128, 0, 8192, 0, 5, 1, 0, 2, 128},
+    {128, 0, 2048, 4, 5, 1, 0, 6, 128},
+    {128, 0, 8192, 0, 5, 1, 0, 6, 128},
     {128, 0, INT64_MAX, 4, 5, 1, 0, 2, 128},
     {128, 1, 2048, 4, 5, 16, 0, 2, 128},
-    {128, 1, 8192, 4, 5, 16, 0, 2, 128},
-    {128, 1, INT64_MAX, 4, 5, 4, 0, 2, 128},
+    {128, 1, 8192, 0, 5, 16, 0, 6, 128},
+    {128, 1, INT64_MAX, 0, 5, 4, 0, 6, 128},
     {64, 0, 2048, 4, 8, 1, 0, 4, 128},
     {64, 0, 8192, 4, 8, 1, 0, 4, 128},
     {64, 0, INT64_MAX, 4, 8, 1, 0, 4, 128},
