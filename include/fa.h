@@ -271,6 +271,8 @@ typedef enum {
  * pointers (FA_ERR_NULL), size limits and multiples of 8 (FA_ERR_SHAPE), alignment
  * (FA_ERR_ALIGN), device (FA_ERR_ARCH / FA_ERR_CUDA).  Arithmetic: bf16 products with fp32
  * accumulation in tensor memory, the epilogue in fp32, C rounded to bf16 (nearest-even).
+ * Problems of more than 128 rows with K > 0 run 256 x 256 tiles on pairs of SMs (a cluster
+ * of two CTAs, tcgen05.mma.cta_group::2); others run 128 x 256 tiles on single SMs.
  * One launch, asynchronous on `stream`; nothing is allocated.
  */
 int fa_gemm(const void* a, const void* b, const void* bias, void* c, int64_t M, int64_t N,
