@@ -235,8 +235,9 @@ int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, in
     int64_t grid = BH * p.n_qtile;
     if (grid > 0x7fffffffLL) return FA_ERR_SHAPE;
     if (sch->alg >= 2) {
-        // two query tiles per CTA
-        grid = BH * ((p.n_qtile + 1) / 2);
+        // two or three query tiles per CTA
+        const int nt = fa::tiles_per_cta(sch->alg);
+        grid = BH * ((p.n_qtile + nt - 1) / nt);
     } else if (sch->persist == 1) {
         // one CTA per SM; causal work comes in units of two query tiles
         const int64_t units = causal ? BH * ((p.n_qtile + 1) / 2) : grid;

@@ -73,10 +73,11 @@
 
 namespace fa {
 
-template <int D, int SLOTS, int BN, bool DB, bool LT>
+template <int D, int SLOTS, int BN, bool DB, bool LT, int NT = 2>
 struct Q2Cfg {
+    static_assert(NT == 2 || NT == 3, "two or three query tiles per CTA");
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
-    static_assert(BN == 64 || BN == 128 || BN == 192, "key tile of 64, 128 or 192 rows");
+    static_assert(BN == 64 || BN == 80 || BN == 128 || BN == 192, "key tile of 64, 80, 128 or 192 rows");
     // with double-buffered scores the issuer needs K_{j+2} while V_j is still
     // unreleased: four loads in flight
     static_assert(SLOTS >= (DB ? 4 : 2), "K/V ring depth");
@@ -86,8 +87,8 @@ struct Q2Cfg {
     static constexpr int kQBoxBytes = 128 * 128;
     static constexpr int kKVBoxBytes = BN * 128;
     static constexpr int kSlots = SLOTS;
-    static constexpr int kQOff = 0;                         // Q_0, then Q_1 (O staging at the end)
-    static constexpr int kSlotOff = 2 * kQTileBytes;
+    static constexpr int kQOff = 0;                         // Q_0, Q_1 (, Q_2) (O staging at the end)
+    static constexpr int kSlotOff = NT * kQTileBytes;
     // LT: a BN-row tile of bf16 ones after the ring; the P.V product reads it as
     // 16 extra columns of V, so O gains 16 columns that each accumulate the sum
     // of the bf16 weights (l^) on the tensor core
@@ -104,28 +105,28 @@ struct Q2Cfg {
     __host__ __device__ static constexpr uint32_t col_s(int ti, int b) {
         return static_cast<uint32_t>((ti * kSBufs + b) * BN);
     }
-    static constexpr uint32_t kColO = 2 * kSBufs * BN;
+    static constexpr uint32_t kColO = NT * kSBufs * BN;
     static constexpr uint32_t kTmemCols = 512;
     static_assert(kSmemBytes <= 232448, "shared memory per CTA (227 KiB)");
-    static_assert(kColO + 2 * kDO <= kTmemCols, "score and output buffers in TMEM");
+    static_assert(kColO + NT * kDO <= kTmemCols, "score and output buffers in TMEM");
     static_assert(kKVBoxBytes % 1024 == 0, "slots on 1024-byte boundaries (128-byte swizzle)");
 };
 
-template <int kSlots>
+template <int kSlots, int NT = 2>
 struct alignas(8) Q2Barriers {
     uint64_t kv_full[kSlots];
     uint64_t kv_empty[kSlots];     // released by one commit after the load's last use
-    uint64_t q_full[2];
-    uint64_t s_full[4];            // [2i + b]: S_i(j) computed into score buffer b
+    uint64_t q_full[NT];
+    uint64_t s_full[2 * NT];       // [2i + b]: S_i(j) computed into score buffer b
     // [2i + b]: the first / second half of P_i(j)'s keys in score buffer b (O_i
     // rescaled before the first), 128 arrivals.  One pair per score buffer:
     // with two buffers the softmax can release P_i(j+1) before the issuer has
     // waited for P_i(j), and a single barrier would then be two phases ahead
     // of that parity wait.
-    uint64_t p_half[4];
-    uint64_t p_full[4];
-    uint64_t pv_done[2];           // O_i += P_i(j) V_j completed (double-buffered scores)
-    uint64_t o_full[2];            // every product of tile i completed
+    uint64_t p_half[2 * NT];
+    uint64_t p_full[2 * NT];
+    uint64_t pv_done[NT];          // O_i += P_i(j) V_j completed (double-buffered scores)
+    uint64_t o_full[NT];           // every product of tile i completed
     uint32_t tmem_base;
     volatile uint32_t abort;
 };
@@ -134,20 +135,26 @@ struct alignas(8) Q2Barriers {
 // taddr and waits until the stores completed.  The fences keep the words fully
 // computed before the asynchronous store and their registers untouched until
 // the wait (neither asm statement tells the compiler that the hardware reads
-// the registers after the store issues).
+// the registers after the store issues).  N is a multiple of 8: 32-column
+// stores, then one of 16 and one of 8 columns for the rest.
 template <int N>
 __device__ __forceinline__ void store_words(uint32_t taddr, uint32_t (&w)[N]) {
-    static_assert(N % 16 == 0, "whole 16-column stores");
+    static_assert(N % 8 == 0, "whole 8-column stores");
+    constexpr int k32 = N / 32, r16 = (N % 32) >= 16 ? 1 : 0, r8 = (N % 16) ? 1 : 0;
+    constexpr int o16 = 32 * k32, o8 = o16 + 16 * r16;
+    const auto fence_all = [&]() {
 #pragma unroll
-    for (int q = 0; q < N / 32; ++q) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&w[32 * q]));
-    if constexpr (N % 32) reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&w[N - 16]));
+        for (int q = 0; q < k32; ++q) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&w[32 * q]));
+        if constexpr (r16) reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&w[o16]));
+        if constexpr (r8) reg_fence8(*reinterpret_cast<uint32_t(*)[8]>(&w[o8]));
+    };
+    fence_all();
 #pragma unroll
-    for (int q = 0; q < N / 32; ++q) tmem_st32(taddr + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&w[32 * q]));
-    if constexpr (N % 32) tmem_st16(taddr + N - 16, *reinterpret_cast<uint32_t(*)[16]>(&w[N - 16]));
+    for (int q = 0; q < k32; ++q) tmem_st32(taddr + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&w[32 * q]));
+    if constexpr (r16) tmem_st16(taddr + o16, *reinterpret_cast<uint32_t(*)[16]>(&w[o16]));
+    if constexpr (r8) tmem_st8(taddr + o8, *reinterpret_cast<uint32_t(*)[8]>(&w[o8]));
     tmem_wait_st();
-#pragma unroll
-    for (int q = 0; q < N / 32; ++q) reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&w[32 * q]));
-    if constexpr (N % 32) reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&w[N - 16]));
+    fence_all();
 }
 
 // Lazy rescale threshold (log2 units): O and the sums are rescaled only when a
@@ -161,13 +168,35 @@ __device__ __forceinline__ void store_words(uint32_t taddr, uint32_t (&w)[N]) {
 // of (warp, key tile) steps.
 constexpr float kRescaleTau = 32.0f;
 
-constexpr int kQ2IssuerWarp = 9;       // issues every tcgen05.mma of the CTA
-constexpr int kQ2AllocWarp = 10;
+// Warp roles and register budgets.  setmaxnreg acts on whole warpgroups (four
+// consecutive warps), so the last warpgroup always holds the producer, the
+// issuer, the TMEM allocator and a spare warp.  Two query tiles: warps 0-7
+// softmax (one per TMEM lane quarter and tile), 8 producer, 9 issuer, 10 TMEM
+// allocation, 11 spare (384 threads launched with 168 registers; the softmax
+// warps raise theirs to 208, the others drop to 88).  Three query tiles: warps
+// 0-11 softmax, 12 producer, 13 issuer, 14 TMEM allocation, 15 spare (512
+// threads launched with 128; softmax 144, the others 80, which also fills each
+// SM partition's 512 registers a lane exactly: three softmax warps and one other).
+template <int NT>
+struct Q2Roles {
+    static constexpr int kSoftWarps = 4 * NT;
+    static constexpr int kProducer = kSoftWarps;
+    static constexpr int kIssuer = kSoftWarps + 1;
+    static constexpr int kAlloc = kSoftWarps + 2;
+    static constexpr int kThreads = 32 * (kSoftWarps + 4);
+    static constexpr int kLaunchRegs = NT == 2 ? 168 : 128;
+    static constexpr uint32_t kRegsSoft = NT == 2 ? kRegsSoftmax : 144;
+    static constexpr uint32_t kRegsRest = NT == 2 ? kRegsOther : 80;
+    static constexpr int kRegTotal = kSoftWarps * 32 * static_cast<int>(kRegsSoft) +
+                                     (kThreads - kSoftWarps * 32) * static_cast<int>(kRegsRest);
+    static_assert(kRegTotal <= kThreads * kLaunchRegs, "register rebalance within the launch");
+    static_assert(kThreads * kLaunchRegs <= 65536, "registers of one SM");
+};
 
-// CTA index -> (b, h) slice and query-tile pair.  Without the mask the pairs
-// of one slice are adjacent in launch order (the slice's K/V stay in L2).
-// Under the mask slices are taken `group` at a time and the pairs of a group
-// launch longest first.
+// CTA index -> (b, h) slice and group of query tiles (a pair, or a triple).
+// Without the mask the groups of one slice are adjacent in launch order (the
+// slice's K/V stay in L2).  Under the mask slices are taken `group` at a time
+// and the tile groups of a slice group launch longest first.
 template <bool CAUSAL>
 __device__ __forceinline__ void map_pair(const FwdParams& p, int n_pair, int id, int& bh, int& c) {
     if constexpr (CAUSAL) {
@@ -183,12 +212,13 @@ __device__ __forceinline__ void map_pair(const FwdParams& p, int n_pair, int id,
     }
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34, int NT>
+__global__ void __launch_bounds__(Q2Roles<NT>::kThreads, 1)
     fa_fwd_2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                      const FwdParams p) {
-    using C = Q2Cfg<D, SLOTS, BN, DB, LT>;
+    using C = Q2Cfg<D, SLOTS, BN, DB, LT, NT>;
+    using R = Q2Roles<NT>;
     // P is released in two parts of kW0 and kW1 words (two keys a word): halves,
     // or with P34 the first three quarters of the keys and then the last quarter.
     // The product with the first part then runs while the last quarter's weights
@@ -196,29 +226,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the key tile's P.V product follows the softmax's last release (instead of
     // half): the chain softmax -> P.V -> next scores -> softmax that bounds a
     // tile's step gets shorter by a quarter of a P.V product.
+    // 80-row key tiles are released as 48 + 32 keys (a 40-key half is not a whole
+    // number of 16-key products)
     static_assert(!P34 || BN == 128, "three-quarter release: key tiles of 128 rows");
-    constexpr int kW0 = P34 ? 3 * BN / 8 : BN / 4;
+    constexpr int kW0 = P34 ? 3 * BN / 8 : (BN == 80 ? 24 : BN / 4);
     constexpr int kW1 = BN / 2 - kW0;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_addr);
-    auto* bars = reinterpret_cast<Q2Barriers<SLOTS>*>(smem + C::kBarOff);
+    auto* bars = reinterpret_cast<Q2Barriers<SLOTS, NT>*>(smem + C::kBarOff);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_pair = (p.n_qtile + 1) / 2;
+    const int n_pair = (p.n_qtile + NT - 1) / NT;     // tile groups per slice
     int bh, c;
     map_pair<CAUSAL>(p, n_pair, blockIdx.x, bh, c);
     const int n_kv_all = (p.N + BN - 1) / BN;
+    // first query row of tile i of this CTA
+    const auto tile_q0 = [&](int i) { return 128 * (NT * c + i); };
     // key tiles of query tile i (0 when the tile lies past N); under the mask
     // the tiles holding keys 0 .. q0+127
     const auto kv_tiles = [&](int i) {
-        const int q0 = 256 * c + 128 * i;
+        const int q0 = tile_q0(i);
         if (q0 >= p.N) return 0;
         return CAUSAL ? min(n_kv_all, (q0 + 128 + BN - 1) / BN) : n_kv_all;
     };
-    const int n_kv = max(kv_tiles(0), kv_tiles(1));
+    int n_kv = 0;
+#pragma unroll
+    for (int i = 0; i < NT; ++i) n_kv = max(n_kv, kv_tiles(i));
 
     const uint32_t bar_kv_full = smem_u32(&bars->kv_full[0]);
     const uint32_t bar_kv_empty = smem_u32(&bars->kv_empty[0]);
@@ -235,12 +271,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar_kv_full + 8 * s, 1);
             mbar_init(bar_kv_empty + 8 * s, 1);
         }
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2 * NT; ++i) {
             mbar_init(bar_s_full + 8 * i, 1);
             mbar_init(bar_p_half + 8 * i, 128);
             mbar_init(bar_p_full + 8 * i, 128);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NT; ++i) {
             mbar_init(bar_q_full + 8 * i, 1);
             mbar_init(bar_pv_done + 8 * i, 1);
             mbar_init(bar_o_full + 8 * i, 1);
@@ -248,22 +284,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         bars->abort = 0u;
         fence_barrier_init();
     }
-    if (warp == kQ2AllocWarp) {
+    if (warp == R::kAlloc) {
         tmem_alloc(smem_u32(&bars->tmem_base), C::kTmemCols);
         tmem_relinquish();
     }
     if constexpr (LT) {
         // the ones tile (bf16 1.0 everywhere, so its swizzled layout needs no care),
-        // written by the 256 softmax threads and made visible to the tensor core
-        if (warp < 8) {
+        // written by the softmax threads and made visible to the tensor core
+        if (warp < R::kSoftWarps) {
             const uint32_t ones = base + C::kOnesOff;
 #pragma unroll 1
-            for (int i = threadIdx.x; i < C::kOnesBytes / 16; i += 256)
+            for (int i = threadIdx.x; i < C::kOnesBytes / 16; i += 32 * R::kSoftWarps)
                 st_shared_v4(ones + 16 * i, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
             fence_proxy_async_smem();
         }
     }
-    if (warp == kProducerWarp && lane == 0) {
+    if (warp == R::kProducer && lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
@@ -274,13 +310,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp < 8) {
-        regs_increase<kRegsSoftmax>();
+    if (warp < R::kSoftWarps) {
+        regs_increase<R::kRegsSoft>();
         // ============================================================ softmax, one row per thread
         const int ti = warp >> 2;                 // query tile of this warpgroup
         const int quarter = warp & 3;
         const int r = 32 * quarter + lane;        // tile row = TMEM lane
-        const int q0 = 256 * c + 128 * ti;
+        const int q0 = tile_q0(ti);
         const int row = q0 + r;
         const int n_i = kv_tiles(ti);
         const uint32_t lane_w = static_cast<uint32_t>(32 * quarter) << 16;
@@ -310,6 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int q = 0; q < n / 32; ++q)
                     tmem_ld32(t_s + c0 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&s[i0 + 32 * q]));
+                if (n % 32)       // 80-row key tiles: 16 more columns
+                    tmem_ld32x16(t_s + c0 + n - 16, *reinterpret_cast<uint32_t(*)[16]>(&s[i0 + n - 16]));
             };
             // after tcgen05.wait::ld: pin s[i0 .. i0+n) after the wait (it carries no
             // register operands) and mask the keys past the row's limit
@@ -317,6 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int q = 0; q < n / 32; ++q)
                     reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(&s[i0 + 32 * q]));
+                if (n % 32) reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(&s[i0 + n - 16]));
                 if (masked) {
 #pragma unroll
                     for (int k = 0; k < n; ++k)
@@ -512,20 +551,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bulk_wait_group_read0();
             }
         }
-    } else if (warp == kProducerWarp) {
-        regs_decrease<kRegsOther>();
+    } else if (warp == R::kProducer) {
+        regs_decrease<R::kRegsRest>();
         // ============================================================ TMA producer
         if (lane == 0) {
             const uint64_t pol_q = policy_evict_first();
             const uint64_t pol_kv = policy_evict_last();
             const uint32_t slot_smem = base + C::kSlotOff;
-            for (int i = 0; i < 2; ++i) {
+            for (int i = 0; i < NT; ++i) {
                 if (kv_tiles(i) == 0) continue;
                 mbar_arrive_expect_tx(bar_q_full + 8 * i, C::kQTileBytes);
 #pragma unroll
                 for (int bx = 0; bx < C::kBoxes; ++bx)
                     tma_load_3d(base + C::kQOff + i * C::kQTileBytes + bx * C::kQBoxBytes, &tm_q, 64 * bx,
-                                256 * c + 128 * i, bh, bar_q_full + 8 * i, pol_q);
+                                tile_q0(i), bh, bar_q_full + 8 * i, pol_q);
             }
             int ld = 0;
             for (int j = 0; j < n_kv; ++j) {
@@ -544,19 +583,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (*abort) {
                 for (int k = max(0, ld - SLOTS); k < ld; ++k)
                     wait_bar(bar_kv_full + 8 * (k % SLOTS), (k / SLOTS) & 1, abort, p.status);
-                for (int i = 0; i < 2; ++i)
+                for (int i = 0; i < NT; ++i)
                     if (kv_tiles(i) > 0) wait_bar(bar_q_full + 8 * i, 0, abort, p.status);
             }
         }
         __syncwarp();
-    } else if (warp == kQ2IssuerWarp) {
-        regs_decrease<kRegsOther>();
+    } else if (warp == R::kIssuer) {
+        regs_decrease<R::kRegsRest>();
         // ============================================================ MMA issuer (both tiles)
         // The whole warp runs the issuing loop (converged, so the descriptor
         // arithmetic stays warp-uniform); one elected lane issues each product
         // and commit.
         {
-            const int n0 = kv_tiles(0), n1 = kv_tiles(1);
+            int n_t[NT];                             // key tiles of each query tile
+#pragma unroll
+            for (int i = 0; i < NT; ++i) n_t[i] = kv_tiles(i);
             const uint32_t slot_smem = base + C::kSlotOff;
             const auto slot_addr = [&](int i) { return slot_smem + (i % SLOTS) * C::kKVTileBytes; };
             // Each ring load (K_j = load 2j, V_j = load 2j+1) is waited for once,
@@ -622,8 +663,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr int kAhead = DB ? 2 : 1;       // score products issued ahead of the softmax
             for (int j = 0; j < kAhead && j < n_kv; ++j) {
                 wait_kv(2 * j);
-                for (int ti = 0; ti < 2; ++ti) {
-                    if (j >= (ti ? n1 : n0)) continue;
+                for (int ti = 0; ti < NT; ++ti) {
+                    if (j >= n_t[ti]) continue;
                     if (j == 0) {
                         wait_bar(bar_q_full + 8 * ti, 0, abort, p.status);
                         tc_fence_after();
@@ -633,8 +674,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit_elect(bar_kv_empty + 8 * ((2 * j) % SLOTS));          // K_j
             }
             for (int j = 0; j < n_kv; ++j) {
-                for (int ti = 0; ti < 2; ++ti) {
-                    const int n_i = ti ? n1 : n0;
+                for (int ti = 0; ti < NT; ++ti) {
+                    const int n_i = n_t[ti];
                     if (j >= n_i) continue;
                     // P_ti(j) sits in score buffer pb; its barriers' phase counts steps on that buffer
                     const int pb = 2 * ti + (DB ? (j & 1) : 0);
@@ -658,17 +699,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_commit_elect(bar_kv_empty + 8 * ((2 * (j + kAhead)) % SLOTS));   // K_{j+kAhead}
             }
             // every product has completed before TMEM is released
-            wait_bar(bar_o_full, 0, abort, p.status);
-            if (n1 > 0) wait_bar(bar_o_full + 8, 0, abort, p.status);
+            for (int i = 0; i < NT; ++i)
+                if (n_t[i] > 0) wait_bar(bar_o_full + 8 * i, 0, abort, p.status);
         }
         __syncwarp();
     } else {
-        regs_decrease<kRegsOther>();   // spare warp of the third warpgroup
+        regs_decrease<R::kRegsRest>();   // spare warp of the third warpgroup
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == kQ2AllocWarp) {
+    if (warp == R::kAlloc) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }

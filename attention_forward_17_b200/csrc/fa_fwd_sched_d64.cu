@@ -23,6 +23,10 @@ const Schedule kD64[] = {
     make_2q_schedule<64, 4, 8, 64, true>(),
     make_2q_schedule<64, 4, 8, 128, false, true>(),
     make_2q_schedule<64, 4, 8, 64, true, true>(), make_2q_schedule<64, 3, 8, 128, false, true>(),
+    make_2q_schedule<64, 4, 8, 64, false, true, false, 3>(), make_2q_schedule<64, 2, 8, 64, false, true, false, 3>(),
+    make_2q_schedule<64, 0, 8, 64, false, true, false, 3>(),
+    make_2q_schedule<64, 4, 8, 80, false, true, false, 3>(), make_2q_schedule<64, 3, 8, 80, false, true, false, 3>(),
+    make_2q_schedule<64, 0, 8, 80, false, true, false, 3>(),
 };
 }  // namespace
 

@@ -31,7 +31,8 @@ struct Schedule {
                        // tile; 3: the same with two score buffers per tile (scores of
                        // the next key tile computed while the softmax works); 4, 5: as
                        // 2, 3 with the sum of the bf16 weights on the tensor core; 6 to 9:
-                       // as 2 to 5 with P released as 3/4 and then 1/4 of the keys
+                       // as 2 to 5 with P released as 3/4 and then 1/4 of the keys; + 8:
+                       // three query tiles per CTA instead of two
     int smem_bytes;    // dynamic shared memory per CTA
     int bn;            // rows of a key/value tile (128 except for the two-query-tile algorithms)
     FwdLaunchFn launch[2];   // [causal]
@@ -83,48 +84,54 @@ constexpr Schedule make_pp_schedule() {
                     &setup_pp_both<D, EMU, SLOTS>};
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34, int NT>
 cudaError_t launch_2q(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                       const CUtensorMap& to, const FwdParams& p, unsigned grid, cudaStream_t stream) {
-    fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN, DB, LT, P34>
-        <<<grid, kThreads, Q2Cfg<D, SLOTS, BN, DB, LT>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+    fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN, DB, LT, P34, NT>
+        <<<grid, Q2Roles<NT>::kThreads, Q2Cfg<D, SLOTS, BN, DB, LT, NT>::kSmemBytes, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
-template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34>
+template <int D, bool CAUSAL, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34, int NT>
 int setup_2q_one() {
-    auto* k = fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN, DB, LT, P34>;
+    auto* k = fa_fwd_2q_kernel<D, CAUSAL, EMU, SLOTS, BN, DB, LT, P34, NT>;
     if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Q2Cfg<D, SLOTS, BN, DB, LT>::kSmemBytes) != cudaSuccess)
+                             Q2Cfg<D, SLOTS, BN, DB, LT, NT>::kSmemBytes) != cudaSuccess)
         return -6;
     cudaFuncAttributes attr;
     if (cudaFuncGetAttributes(&attr, k) != cudaSuccess) return -6;
-    if (attr.numRegs * kThreads < kRegSplitTotal) return -6;
+    if (attr.numRegs * Q2Roles<NT>::kThreads < Q2Roles<NT>::kRegTotal) return -6;
     return 0;
 }
 
-template <int D, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34>
+template <int D, int EMU, int SLOTS, int BN, bool DB, bool LT, bool P34, int NT>
 int setup_2q_both() {
-    const int rc = setup_2q_one<D, false, EMU, SLOTS, BN, DB, LT, P34>();
-    return rc ? rc : setup_2q_one<D, true, EMU, SLOTS, BN, DB, LT, P34>();
+    const int rc = setup_2q_one<D, false, EMU, SLOTS, BN, DB, LT, P34, NT>();
+    return rc ? rc : setup_2q_one<D, true, EMU, SLOTS, BN, DB, LT, P34, NT>();
 }
 
-// Two query tiles per CTA (fa_fwd_2q_kernel), key tiles of BN rows: algorithm
-// 2 (one score buffer per tile), + 1 with two score buffers per tile (DB), + 2
-// with the sum of the bf16 weights accumulated by the tensor core (LT), + 4 with
-// P released as three quarters and one quarter of the keys (P34): 2 to 9.
-template <int D, int EMU, int SLOTS, int BN = 128, bool DB = false, bool LT = false, bool P34 = false>
+// Several query tiles per CTA (fa_fwd_2q_kernel), key tiles of BN rows:
+// algorithm 2 (two query tiles, one score buffer per tile), + 1 with two score
+// buffers per tile (DB), + 2 with the sum of the bf16 weights accumulated by the
+// tensor core (LT), + 4 with P released as three quarters and one quarter of the
+// keys (P34), + 8 with three query tiles per CTA (NT = 3).
+template <int D, int EMU, int SLOTS, int BN = 128, bool DB = false, bool LT = false, bool P34 = false,
+          int NT = 2>
 constexpr Schedule make_2q_schedule() {
     return Schedule{D,
                     EMU,
                     SLOTS,
                     0,
-                    2 + (DB ? 1 : 0) + (LT ? 2 : 0) + (P34 ? 4 : 0),
-                    Q2Cfg<D, SLOTS, BN, DB, LT>::kSmemBytes,
+                    2 + (DB ? 1 : 0) + (LT ? 2 : 0) + (P34 ? 4 : 0) + (NT == 3 ? 8 : 0),
+                    Q2Cfg<D, SLOTS, BN, DB, LT, NT>::kSmemBytes,
                     BN,
-                    {&launch_2q<D, false, EMU, SLOTS, BN, DB, LT, P34>, &launch_2q<D, true, EMU, SLOTS, BN, DB, LT, P34>},
-                    &setup_2q_both<D, EMU, SLOTS, BN, DB, LT, P34>};
+                    {&launch_2q<D, false, EMU, SLOTS, BN, DB, LT, P34, NT>,
+                     &launch_2q<D, true, EMU, SLOTS, BN, DB, LT, P34, NT>},
+                    &setup_2q_both<D, EMU, SLOTS, BN, DB, LT, P34, NT>};
 }
+
+// Query tiles per CTA of a schedule's algorithm.
+constexpr int tiles_per_cta(int alg) { return alg < 2 ? 1 : (((alg - 2) & 8) ? 3 : 2); }
 
 template <int D, bool CAUSAL, int EMU, int SLOTS, int PERSIST>
 cudaError_t launch_schedule(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

@@ -212,10 +212,9 @@ def write_report(rows, table, device_name, path, top=6):
            "round's timed launches; per GHz = TFLOP/s / (MHz / 1000); reasons = clock-event reasons "
            "seen. `ok` = output within twice the oracle's parity bars of the default schedule's (each "
            "is held to the oracle's bars by the parity tests). alg: 0 one "
-           "query tile per CTA, 1 split-KV ping-pong, 2 two query tiles per CTA, 3 two query tiles with "
-           "two score buffers each, 4 and 5 as 2 and 3 with the bf16 weight sums on the tensor core, 6 to 9 as 2 to 5 "
-           "with P released as 3/4 and 1/4 of the keys; "
-           "launch: 0 one CTA "
+           "query tile per CTA, 1 split-KV ping-pong, 2 two query tiles per CTA, then + 1 two score buffers "
+           "per tile, + 2 bf16 weight sums on the tensor core, + 4 P released as 3/4 and 1/4 of the keys, "
+           "+ 8 three query tiles per CTA; launch: 0 one CTA "
            "per tile, 1 static persistent, 2 cluster launch control.", ""]
     keys = []
     for r in rows:

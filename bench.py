@@ -47,6 +47,7 @@ WORKLOADS = {
     "b1_h32_n16384_d128": dict(B=1, H=32, N=16384, d=128, sigma_qk=1.0),
     "b2_h16_n4096_d128": dict(B=2, H=16, N=4096, d=128, sigma_qk=1.0),
     "b1_h32_n16384_d64": dict(B=1, H=32, N=16384, d=64, sigma_qk=1.0),
+    "b4_h16_n4096_d64": dict(B=4, H=16, N=4096, d=64, sigma_qk=1.0),
     "b4_h8_n1024_d64": dict(B=4, H=8, N=1024, d=64, sigma_qk=1.0),
     # profiling size: Q, K, V, O = 4 x 64 MiB, above the L2, a short launch
     "b1_h64_n4096_d128": dict(B=1, H=64, N=4096, d=128, sigma_qk=1.0),
@@ -71,7 +72,7 @@ def load_peaks():
         return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
 
 
-KERNEL_FAMILY = {0: "fa_fwd_kernel", 1: "fa_fwd_pp_kernel", **{a: "fa_fwd_2q_kernel" for a in range(2, 10)}}
+KERNEL_FAMILY = {0: "fa_fwd_kernel", 1: "fa_fwd_pp_kernel", **{a: "fa_fwd_2q_kernel" for a in range(2, 18)}}
 
 
 def measured_traffic(workload, algorithm=0):

@@ -134,7 +134,9 @@ int fa_fwd_status(const void* q, const void* k, const void* v, void* o, float* l
  *                     the sum of the bf16 weights accumulated by the tensor
  *                     core, d = 64 only; 6 to 9 = as 2 to 5 with P released
  *                     to the tensor core as the first three quarters and then
- *                     the last quarter of a 128-key tile), shared memory per CTA
+ *                     the last quarter of a 128-key tile; + 8 = three query
+ *                     tiles per CTA instead of two, d = 64 only), shared memory
+ *                     per CTA
  *                     and rows of a key/value tile (128, or 64 / 192 for some
  *                     two-tile schedules) of schedule `id`; FA_ERR_ARG for an
  *                     unknown id.  Output pointers may be NULL.
@@ -167,8 +169,8 @@ int fa_fwd_schedule(const void* q, const void* k, const void* v, void* o, float*
  *   dev_counts   device, two unsigned 64-bit counters, caller-owned, never
  *                cleared: [0] += (warp, key tile) steps at which at least one
  *                of the warp's 32 rows rescaled, [1] += (row, key tile)
- *                rescales.  Only the two-query-tile kernel (algorithms 2
- *                to 9) counts; other schedules leave the counters unchanged.
+ *                rescales.  Only the multi-tile kernel (algorithms 2
+ *                and above) counts; other schedules leave the counters unchanged.
  *                NULL -> FA_ERR_NULL (after the checks of fa_fwd).
  * A diagnostic entry point: the atomics cost a little time.
  */

@@ -150,16 +150,18 @@ def test_schedule_registry():
     for i in range(n):
         assert LIB.fa_schedule_info(i, *[ctypes.byref(x) for x in vals]) == fa.FA_OK
         d, emu, slots, persist, alg, smem, bn = (x.value for x in vals)
-        # key tiles of 128 rows, or 64 / 192 for the two-tile kernel where two
-        # score and two output buffers fit the 512 TMEM columns
-        # two-tile algorithms: 2 + (1: two score buffers) + (2: l^ on the tensor core)
+        # key tiles of 128 rows, or 64 / 192 for the multi-tile kernel where the
+        # score and output buffers of its query tiles fit the 512 TMEM columns
+        # multi-tile algorithms: 2 + (1: two score buffers) + (2: l^ on the tensor core)
         # + (4: P released as three quarters and one quarter of the keys)
+        # + (8: three query tiles per CTA instead of two)
         bits = alg - 2 if alg >= 2 else 0
         bufs = 2 if bits & 1 else 1           # score buffers per query tile
         do = d + 16 if bits & 2 else d        # O columns (16 more when the tensor core sums l^)
-        assert 2 * bufs * bn + 2 * do <= 512 and (bn == 128 or (alg >= 2 and bn in (64, 192)))
+        nt = 3 if bits & 8 else 2             # query tiles per CTA
+        assert nt * (bufs * bn + do) <= 512 and (bn == 128 or (alg >= 2 and bn in (64, 80, 192)))
         assert d in (64, 128) and emu in (0, 2, 3, 4, 8) and persist in (0, 1, 2)
-        assert alg in range(10) and 0 < smem <= 232448
+        assert alg in range(18) and 0 < smem <= 232448
         assert not (bits & 4) or bn == 128     # the three-quarter release needs 128-row key tiles
         # the one-tile kernels need four slots for sound parity waits; the
         # two-tile kernel's issuers observe every load in order, so any depth >= 2

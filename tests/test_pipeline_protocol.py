@@ -137,9 +137,10 @@ def test_model_flags_an_odd_ring_for_the_ping_pong_kernel():
 
 
 # ------------------------------------------------------------------ two-query-tile kernel
-def two_tile_issuer_events(n0, n1, ahead=1, release_k_early=False):
-    """The ring events of the two-query-tile kernel's MMA issuer, in program
-    order, for key-tile counts n0 (tile 0) and n1 (tile 1): ("wait", L),
+def two_tile_issuer_events(n0, n1, ahead=1, release_k_early=False, more=()):
+    """The ring events of the multi-tile kernel's MMA issuer, in program
+    order, for key-tile counts n0 (tile 0), n1 (tile 1) and `more` (further
+    tiles of a CTA that holds three): ("wait", L),
     ("use", L), ("release", L) with L the load index (K_j = 2j, V_j = 2j+1).
     `ahead` is how many score products run ahead of the softmax (1 with one
     score buffer per tile, 2 with two).  release_k_early models a faulty
@@ -151,15 +152,16 @@ def two_tile_issuer_events(n0, n1, ahead=1, release_k_early=False):
             waited[0] += 1
             ev.append(("wait", waited[0]))
 
-    n_kv = max(n0, n1)
+    counts = (n0, n1) + tuple(more)
+    n_kv = max(counts)
     for j in range(min(ahead, n_kv)):
         wait(2 * j)
-        for n_i in (n0, n1):
+        for n_i in counts:
             if j < n_i:
                 ev.append(("use", 2 * j))
         ev.append(("release", 2 * j))
     for j in range(n_kv):
-        for ti, n_i in ((0, n0), (1, n1)):
+        for ti, n_i in enumerate(counts):
             if j >= n_i:
                 continue
             wait(2 * j + 1)
@@ -204,21 +206,35 @@ def two_tile_violations(n0, n1, slots, **kw):
 
 
 def compiled_two_tile_rings():
-    """(depth, score products ahead) of every compiled two-tile schedule."""
-    return sorted({(s["kv_slots"], 2 if (s["algorithm"] - 2) & 1 else 1)
+    """(depth, score products ahead, query tiles per CTA) of every compiled
+    multi-tile schedule."""
+    return sorted({(s["kv_slots"], 2 if (s["algorithm"] - 2) & 1 else 1, 3 if (s["algorithm"] - 2) & 8 else 2)
                    for s in fa.schedules() if s["algorithm"] >= 2})
 
 
-@pytest.mark.parametrize("slots,ahead", compiled_two_tile_rings())
-def test_two_tile_ring_is_sound(slots, ahead):
-    for n1 in range(0, 40):
-        # non-causal (equal counts), causal (tile 0 one to three key tiles short,
-        # for key tiles of 192, 128 and 64 rows), and a second tile past the end
-        # of the sequence (no keys)
-        for n0 in {n1, n1 - 1, n1 - 2}:
-            if n0 >= 1:
-                assert two_tile_violations(n0, n1, slots, ahead=ahead) == 0, (n0, n1)
-        assert two_tile_violations(n1 + 1, 0, slots, ahead=ahead) == 0
+@pytest.mark.parametrize("slots,ahead,nt", compiled_two_tile_rings())
+def test_two_tile_ring_is_sound(slots, ahead, nt):
+    for n in range(0, 40):
+        if nt == 2:
+            # non-causal (equal counts), causal (tile 0 one to three key tiles short,
+            # for key tiles of 192, 128 and 64 rows), and a second tile past the end
+            # of the sequence (no keys)
+            for n0 in {n, n - 1, n - 2}:
+                if n0 >= 1:
+                    assert two_tile_violations(n0, n, slots, ahead=ahead) == 0, (n0, n)
+            assert two_tile_violations(n + 1, 0, slots, ahead=ahead) == 0
+        else:
+            # three tiles: equal counts, causal steps of one or two key tiles per
+            # query tile, and the last one or two tiles past the end
+            for step in (0, 1, 2):
+                if n - 2 * step >= 1:
+                    assert two_tile_violations(n - 2 * step, n - step, slots, ahead=ahead, more=(n,)) == 0
+            assert two_tile_violations(n + 1, n + 1, slots, ahead=ahead, more=(0,)) == 0
+            assert two_tile_violations(n + 1, 0, slots, ahead=ahead, more=(0,)) == 0
+
+
+def test_three_tile_schedules_exist():
+    assert any((s["algorithm"] - 2) & 8 for s in fa.schedules() if s["algorithm"] >= 2)
 
 
 def test_model_flags_a_shallow_ring_with_two_score_buffers():

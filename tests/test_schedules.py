@@ -70,9 +70,9 @@ def test_persistent_walks_every_tile(cuda_device, d, N):
 
 @pytest.mark.gpu
 def test_two_tile_kernel_edges(cuda_device):
-    # the two-query-tile kernel on shapes that exercise its pairing: one row, a
-    # lone first tile, a pair whose second tile is ragged or empty (odd tile
-    # counts), several slices, both masks
+    # the multi-tile kernel on shapes that exercise its grouping of query tiles
+    # (pairs, or triples): one row, a lone first tile, a group whose last tiles
+    # are ragged or empty, several slices, both masks
     sched = [s for s in _schedules() if s["algorithm"] >= 2]
     assert sched, "no two-query-tile schedule compiled"
     for s in sched:
