@@ -224,7 +224,7 @@ def test_schedule_table_entries_are_compiled():
     import re
     import os
     path = os.path.join(os.path.dirname(fa.LIB_PATH), "csrc", "fa_schedule_table.h")
-    rows = re.findall(r"\{(\d+), (\d), (\w+), (\d), (\d), (\d+), (\d), (\d), (\d+)\},", open(path).read())
+    rows = re.findall(r"\{(\d+), (\d), (\w+), (\d+), (\d+), (\d+), (\d), (\d+), (\d+)\},", open(path).read())
     assert rows, "no table rows parsed"
     compiled = {(s["d"], s["emu_every"], s["kv_slots"], s["persistent"], s["algorithm"], s["key_tile"])
                 for s in fa.schedules()}
