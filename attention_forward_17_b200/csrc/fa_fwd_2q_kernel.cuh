@@ -1,4 +1,4 @@
-// Two-query-tile variant of the fused attention forward pass for sm_100a.
+// Multi-query-tile variant of the fused attention forward pass for sm_100a.
 //
 // Same operation, inputs, outputs and host interface as fa_fwd_kernel (the
 // FlashAttention forward pass of the "TileLang tutorial": query, key and value
@@ -6,9 +6,11 @@
 // normalisation sums and rescaling factors, both products on the tensor
 // cores).  What differs is the work unit: a CTA owns TWO 128-row query tiles
 // of one (b, h) slice (rows 256c .. 256c+255) and streams every key/value tile
-// once for both of them.
+// once for both of them.  At d = 64 a CTA may own THREE (NT = 3, rows 384c ..
+// 384c+383): the description below is for two, and three tiles extend every
+// per-tile role, barrier and buffer by one (see Q2Roles for the warps).
 //
-// Roles (384 threads):
+// Roles (384 threads with two tiles):
 //   warps 0-3  softmax for query tile 0, warps 4-7 for query tile 1.  A thread
 //              owns one query row (TMEM lane = row, 32x32b accesses): a row's
 //              scores of a key tile pass through one thread's registers, so
@@ -23,10 +25,10 @@
 //              the 64 the tensor core needs for one).
 //   warp 10    allocates and frees TMEM.
 //
-// Key tiles are BN rows (BN = 64, 128 or 192, a template parameter; the tile
-// of queries is always 128 rows).  Tensor memory (512 columns): S_0 [0,BN),
+// Key tiles are BN rows (BN = 64, 80, 128 or 192, a template parameter; the
+// tile of queries is always 128 rows).  Tensor memory (512 columns): S_0 [0,BN),
 // S_1 [BN,2BN), O_0 [2BN,2BN+D), O_1 [2BN+D,2BN+2D), which bounds BN by
-// 2 BN + 2 D <= 512.  The softmax writes P_i (bf16, two keys per column) over
+// 2 BN + 2 D <= 512 (NT BN + NT D <= 512 with NT tiles).  The softmax writes P_i (bf16, two keys per column) over
 // the first BN/2 columns of S_i once it has read them, and O_i += P_i V_j reads
 // P_i straight from TMEM (the tensor core's TMEM-A form), so P never touches
 // shared memory.
