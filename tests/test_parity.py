@@ -101,6 +101,17 @@ def test_b1_h32_n16384_d128_wide_whole(cuda_device, sigma, causal):
     whole_case(1, 32, 16384, 128, causal, sigma=sigma)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_d64_default_path_whole(cuda_device, causal):
+    # d = 64 at a length where the table picks three query tiles per CTA: 40
+    # query tiles per slice, so the last tile group holds a lone tile, and the
+    # wide score range
+    import attention_forward_17_b200 as fa
+    sid, _ = fa.pick_schedule(5000, 64, causal)
+    print("schedule", fa.schedules()[sid])
+    whole_case(2, 8, 5000, 64, causal, sigma=3.0)
+
+
 def test_b2_h16_n4096_d128_causal(cuda_device):
     sampled_case(2, 16, 4096, 128, True)
 
