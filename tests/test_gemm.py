@@ -48,6 +48,8 @@ SHAPES = [
     (300, 520, 200),     # ragged M, N (last column block is 8 wide), K (last block 8 deep)
     (257, 264, 72),
     (129, 136, 24),      # one 256-row pair tile: the second CTA holds a single valid row
+    (300, 8, 8),         # pair tiles whose second CTA's columns of B all lie past N
+    (520, 24, 1032),     # 17 K blocks, the last 8 deep, on a two-block pair grid
     (640, 768, 1024),    # 16 K blocks: the stage rings wrap several times
 ]
 
